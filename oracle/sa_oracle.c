@@ -1,0 +1,402 @@
+/*
+ * sa_oracle.c -- CPU oracle for the SageAttention-style low-bit attention forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library and its
+ * Python binding) may include, link, load or call this file.  Only the test-suite,
+ * the smoke check and the CPU-baseline leg of the benchmark use it.  It shares no
+ * code, header, table or constant generator with the CUDA path.
+ *
+ * Plain, slow, single-threaded C11.  Build with
+ *     gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fPIC -shared
+ * so that every float operation is one IEEE-754 binary32 (or binary64) operation
+ * rounded to nearest-even, in the order written (x86-64 SSE arithmetic, no FMA
+ * contraction, no re-association).
+ *
+ * What the method computes (sources, by page and section):
+ *   - "AIGC weekend special 5.10: full-stack optimisation of visual-generation
+ *     inference", section 1 (TurboDiffusion), 1.2 Method, item (1): SageAttention2++
+ *     quantises Q and K to low bit (INT4/INT8) and runs Q.K^T on tensor cores; item (2):
+ *     SLA sparse attention runs on top of it.
+ *   - "Video-Generation-101: inference systems", kernel paragraph: SageAttention2 is a
+ *     co-design of number format, thread granularity and accumulation; reference [3]
+ *     names "thorough outlier smoothing".
+ *   - "Video-Generation-101 research log", section 5.5 table, SageAttention2 row:
+ *     INT4/INT8 Q.K^T, FP8/FP16 P.V.
+ *   - NetEase article on the TurboDiffusion release, "attention acceleration" section:
+ *     SageAttention2++ variant; SLA keeps "critical" blocks of the attention weights
+ *     (figure caption).
+ *   - FlashAttention (IO-aware tiled attention, same digest's timeline, 2022.06):
+ *     online softmax over key blocks.
+ * The pages give the outline only; the numerical definition implemented here is:
+ *   K smoothed by subtracting its per-channel mean over tokens; Q quantised to INT8 per
+ *   128-token block and K per 64-token block with scale = max|x|/127 and round-half-even;
+ *   S = q_i8 . k_i8^T exact in int32, dequantised by scale_q * scale_k * sm_scale;
+ *   online softmax in fp32; P scaled by 448 and cast to FP8 e4m3; V cast to FP8 e4m3
+ *   per channel with scale = max|v|/448; P.V accumulated in fp32.
+ * Readings where the pages are silent are marked "reading:" below.
+ *
+ * Parity pins (tests/test_oracle_*.py): e4m3 codec against the OCP FP8 definition and
+ * a library cast; quantiser closed forms (exact-integer case, tie cases, block
+ * boundaries, shift invariance); attention closed forms (N = 1, identical keys,
+ * dominant key), invariants (rows sum to one, constant V columns), brute force against
+ * the fp64 exact attention below.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define QBLK 128 /* query tokens per quantisation block and per mask row */
+#define KBLK 64  /* key tokens per quantisation block and per mask column */
+
+static int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+static int64_t padded_len(int64_t n) { return cdiv64(n, QBLK) * QBLK; }
+
+static float bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------------------------
+ * FP8 e4m3 (OCP 8-bit floating point specification, E4M3 variant): 1 sign bit, 4
+ * exponent bits with bias 7, 3 mantissa bits.  No infinities; exponent 1111 with
+ * mantissa 111 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.  Exponent
+ * field 0 holds subnormals m/8 * 2^-6 = m * 2^-9.
+ * ---------------------------------------------------------------------------------- */
+
+/* Magnitude of the non-negative code c (0..126), exactly, as a double. */
+static double e4m3_magnitude(int c)
+{
+    int e = (c >> 3) & 15;
+    int m = c & 7;
+    if (e == 0) return ldexp((double)m, -9);
+    return ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+}
+
+float sa_oracle_e4m3_to_f32(uint8_t b)
+{
+    int mag = b & 0x7F;
+    if (mag == 0x7F) return NAN;
+    double v = e4m3_magnitude(mag);
+    return (float)((b & 0x80) ? -v : v);
+}
+
+/* Round to nearest, ties to the even code, saturating to +-448 ("satfinite").
+ * reading: values at or beyond the largest finite magnitude clamp to it; NaN maps
+ * to the NaN code (never reached from finite inputs). */
+uint8_t sa_oracle_e4m3_from_f32(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    /* largest code lo in [0,126] whose magnitude is <= a (codes increase with value) */
+    int lo = 0, hi = 126;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (e4m3_magnitude(mid) <= a) lo = mid; else hi = mid - 1;
+    }
+    if (e4m3_magnitude(lo) == a) return (uint8_t)(sign | lo);
+    int up = lo + 1; /* magnitude(up) > a and up <= 126 because a < 448 */
+    double dlo = a - e4m3_magnitude(lo);
+    double dup = e4m3_magnitude(up) - a;
+    int c;
+    if (dlo < dup) c = lo;
+    else if (dup < dlo) c = up;
+    else c = (lo % 2 == 0) ? lo : up; /* tie: the code whose mantissa LSB is 0 */
+    return (uint8_t)(sign | c);
+}
+
+/* ------------------------------------------------------------------------------------
+ * INT8 code of x under scale s: round-half-even of the IEEE quotient x/s, clamped to
+ * [-127, 127].  reading: the quotient is an IEEE fp32 division (not x * (1/s)); a zero
+ * scale (all-zero block) gives code 0.
+ * ---------------------------------------------------------------------------------- */
+static int8_t int8_code(float x, float s)
+{
+    if (s == 0.0f) return 0;
+    float r = nearbyintf(x / s); /* FE_TONEAREST: ties to even */
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/* Per-channel mean of one head's K over its N tokens.
+ * reading: the sum runs in fp64 over t = 0..N-1 in order, is divided by N in fp64 and
+ * rounded once to fp32.  *all_exact is cleared when some channel's fp64 running sum was
+ * not exact (checked with Knuth's TwoSum error term), i.e. when another summation order
+ * could give a different fp64 sum. */
+static void k_mean_head(const uint16_t *k, int64_t N, int d, float *mean, int *all_exact)
+{
+    for (int c = 0; c < d; ++c) {
+        double s = 0.0;
+        int exact = 1;
+        for (int64_t t = 0; t < N; ++t) {
+            double x = (double)bf16_to_f32(k[t * d + c]);
+            double sum = s + x;
+            /* TwoSum: err is the exact rounding error of s + x */
+            double bp = sum - s;
+            double ap = sum - bp;
+            double err = (s - ap) + (x - bp);
+            if (err != 0.0) exact = 0;
+            s = sum;
+        }
+        mean[c] = (float)(s / (double)N);
+        if (!exact) *all_exact = 0;
+    }
+}
+
+/* Q: per (b,h) and 128-token block i, scale_q = max|q|/127 over the block's valid
+ * tokens and all channels; q_i8 = code(q, scale_q).  K: smoothed ks = k - mean_k[c]
+ * (one fp32 subtraction), then per 64-token block scale_k = max|ks|/127 and
+ * k_i8 = code(ks, scale_k).  Rows from N up to the padded length are zero.
+ * Layouts: q,k bf16 [B,H,N,d]; q_i8,k_i8 [B,H,Npad,d]; q_scale [B,H,nq];
+ * k_scale [B,H,nk]; k_mean [B,H,d].  Returns 1 when every K mean came from an exact
+ * fp64 sum, else 0. */
+int sa_oracle_quantize_qk(const uint16_t *q, const uint16_t *k, int B, int H, int N, int d,
+                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                          float *k_mean)
+{
+    fesetround(FE_TONEAREST);
+    const int64_t Npad = padded_len(N);
+    const int64_t nq = cdiv64(N, QBLK), nk = cdiv64(N, KBLK);
+    int all_exact = 1;
+    float *ks = (float *)malloc(sizeof(float) * (size_t)N * (size_t)d);
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        const uint16_t *qh = q + bh * N * d;
+        const uint16_t *kh = k + bh * N * d;
+        int8_t *q8 = q_i8 + bh * Npad * d;
+        int8_t *k8 = k_i8 + bh * Npad * d;
+        memset(q8, 0, (size_t)(Npad * d));
+        memset(k8, 0, (size_t)(Npad * d));
+
+        for (int64_t i = 0; i < nq; ++i) {
+            int64_t t0 = i * QBLK, t1 = t0 + QBLK < N ? t0 + QBLK : N;
+            float amax = 0.0f;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int c = 0; c < d; ++c) {
+                    float a = fabsf(bf16_to_f32(qh[t * d + c]));
+                    if (a > amax) amax = a;
+                }
+            float s = amax / 127.0f;
+            q_scale[bh * nq + i] = s;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int c = 0; c < d; ++c)
+                    q8[t * d + c] = int8_code(bf16_to_f32(qh[t * d + c]), s);
+        }
+
+        float *mean = k_mean + bh * d;
+        k_mean_head(kh, N, d, mean, &all_exact);
+        for (int64_t t = 0; t < N; ++t)
+            for (int c = 0; c < d; ++c)
+                ks[t * d + c] = bf16_to_f32(kh[t * d + c]) - mean[c];
+
+        for (int64_t j = 0; j < nk; ++j) {
+            int64_t t0 = j * KBLK, t1 = t0 + KBLK < N ? t0 + KBLK : N;
+            float amax = 0.0f;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int c = 0; c < d; ++c) {
+                    float a = fabsf(ks[t * d + c]);
+                    if (a > amax) amax = a;
+                }
+            float s = amax / 127.0f;
+            k_scale[bh * nk + j] = s;
+            for (int64_t t = t0; t < t1; ++t)
+                for (int c = 0; c < d; ++c)
+                    k8[t * d + c] = int8_code(ks[t * d + c], s);
+        }
+    }
+    free(ks);
+    return all_exact;
+}
+
+/* V: per (b,h) and channel c, scale_v = max_t |v|/448 over all N tokens;
+ * v_fp8 = e4m3(v / scale_v), stored transposed as [B,H,d,Npad] (channel-major, keys
+ * contiguous), padded keys zero.  reading: per-channel scale over the whole sequence;
+ * the quotient is an IEEE fp32 division; a zero scale gives code 0. */
+void sa_oracle_quantize_v(const uint16_t *v, int B, int H, int N, int d, uint8_t *v_fp8_t,
+                          float *v_scale)
+{
+    fesetround(FE_TONEAREST);
+    const int64_t Npad = padded_len(N);
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        const uint16_t *vh = v + bh * N * d;
+        uint8_t *vt = v_fp8_t + bh * d * Npad;
+        memset(vt, 0, (size_t)(d * Npad));
+        for (int c = 0; c < d; ++c) {
+            float amax = 0.0f;
+            for (int64_t t = 0; t < N; ++t) {
+                float a = fabsf(bf16_to_f32(vh[t * d + c]));
+                if (a > amax) amax = a;
+            }
+            float s = amax / 448.0f;
+            v_scale[bh * d + c] = s;
+            for (int64_t t = 0; t < N; ++t)
+                vt[c * Npad + t] = (s == 0.0f) ? 0 : sa_oracle_e4m3_from_f32(bf16_to_f32(vh[t * d + c]) / s);
+        }
+    }
+}
+
+/* Kept 64-key blocks of query block i, ascending.  mask is [B,H,nq,nk] uint8 with
+ * nonzero = keep, or NULL (every block kept).  Returns the count. */
+static int64_t kept_blocks(const uint8_t *mask, int64_t bh, int64_t i, int64_t nq, int64_t nk,
+                           int64_t *out)
+{
+    int64_t n = 0;
+    for (int64_t j = 0; j < nk; ++j)
+        if (!mask || mask[(bh * nq + i) * nk + j]) out[n++] = j;
+    return n;
+}
+
+/* Quantised attention for selected query rows.
+ * rows: nrows pairs (bh, r) flattened as int64 [2*nrows]; out: fp32 [nrows, d].
+ * group: how many kept 64-key blocks form one online-softmax step (1 or 2).
+ *   reading: the pages fix the online softmax but not its step; steps are runs of
+ *   `group` consecutive kept blocks in ascending order (the last run may be shorter).
+ * Per step, for the step's keys t (t < N):
+ *   S_t = sum_c q_i8[r,c] * k_i8[t,c]                 (int32, exact)
+ *   s_t = (float)S_t * (scale_q[i] * scale_k[j(t)] * sm_scale)   (fp32, left to right)
+ *   m'  = max(m, max_t s_t);  alpha = exp(m - m') (0 while m = -inf)
+ *   p8_t = e4m3(448 * exp(s_t - m'))                  (decoded to fp32)
+ *   l   = alpha * l + sum_t p8_t
+ *   acc = alpha * acc + sum_t p8_t * v_fp8[t,c]       (fp32, keys ascending)
+ * then O[r,c] = acc[c] * scale_v[c] / l, or 0 when l = 0 (no kept key).
+ * reading: l sums the FP8-rounded P, the same weights that multiply V, so a constant V
+ * column is reproduced and the normalised weights sum to one up to fp32 rounding.
+ * reading: alpha is applied whenever the running max grows (no lazy rescaling, which
+ * would push 448*P past the e4m3 range). */
+void sa_oracle_attn_rows(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                         const float *k_scale, const uint8_t *v_fp8_t, const float *v_scale,
+                         int B, int H, int N, int d, float sm_scale, const uint8_t *mask,
+                         int group, const int64_t *rows, int64_t nrows, float *out)
+{
+    fesetround(FE_TONEAREST);
+    (void)B; (void)H;
+    const int64_t Npad = padded_len(N);
+    const int64_t nq = cdiv64(N, QBLK), nk = cdiv64(N, KBLK);
+    int64_t *blocks = (int64_t *)malloc(sizeof(int64_t) * (size_t)nk);
+    float *s = (float *)malloc(sizeof(float) * (size_t)(KBLK * (group > 0 ? group : 1)));
+    int64_t *tk = (int64_t *)malloc(sizeof(int64_t) * (size_t)(KBLK * (group > 0 ? group : 1)));
+    float *acc = (float *)malloc(sizeof(float) * (size_t)d);
+    float *blk = (float *)malloc(sizeof(float) * (size_t)d);
+    if (group < 1) group = 1;
+
+    for (int64_t n = 0; n < nrows; ++n) {
+        const int64_t bh = rows[2 * n], r = rows[2 * n + 1];
+        const int64_t i = r / QBLK;
+        const int8_t *qrow = q_i8 + (bh * Npad + r) * d;
+        const int8_t *kh = k_i8 + bh * Npad * d;
+        const uint8_t *vt = v_fp8_t + bh * d * Npad;
+        const float sq = q_scale[bh * nq + i];
+        const int64_t nkept = kept_blocks(mask, bh, i, nq, nk, blocks);
+
+        float m = -INFINITY, l = 0.0f;
+        for (int c = 0; c < d; ++c) acc[c] = 0.0f;
+
+        for (int64_t g0 = 0; g0 < nkept; g0 += group) {
+            int64_t g1 = g0 + group < nkept ? g0 + group : nkept;
+            int64_t nt = 0;
+            float bmax = -INFINITY;
+            for (int64_t g = g0; g < g1; ++g) {
+                const int64_t j = blocks[g];
+                const float sk = k_scale[bh * nk + j];
+                for (int64_t t = j * KBLK; t < (j + 1) * KBLK && t < N; ++t) {
+                    int32_t S = 0;
+                    for (int c = 0; c < d; ++c) S += (int32_t)qrow[c] * (int32_t)kh[t * d + c];
+                    float sc = sq * sk;
+                    sc = sc * sm_scale;
+                    s[nt] = (float)S * sc;
+                    tk[nt] = t;
+                    if (s[nt] > bmax) bmax = s[nt];
+                    ++nt;
+                }
+            }
+            if (nt == 0) continue;
+            const float mnew = m > bmax ? m : bmax;
+            const float alpha = (m == -INFINITY) ? 0.0f : expf(m - mnew);
+            float psum = 0.0f;
+            for (int c = 0; c < d; ++c) blk[c] = 0.0f;
+            for (int64_t u = 0; u < nt; ++u) {
+                float p = expf(s[u] - mnew);
+                float p8 = sa_oracle_e4m3_to_f32(sa_oracle_e4m3_from_f32(448.0f * p));
+                psum += p8;
+                for (int c = 0; c < d; ++c)
+                    blk[c] += p8 * sa_oracle_e4m3_to_f32(vt[(int64_t)c * Npad + tk[u]]);
+            }
+            l = alpha * l + psum;
+            for (int c = 0; c < d; ++c) acc[c] = alpha * acc[c] + blk[c];
+            m = mnew;
+        }
+        float *o = out + n * d;
+        for (int c = 0; c < d; ++c) {
+            const float sv = v_scale[bh * d + c];
+            o[c] = (l > 0.0f) ? (acc[c] * sv) / l : 0.0f;
+        }
+    }
+    free(blocks); free(s); free(tk); free(acc); free(blk);
+}
+
+/* Exact attention in fp64 for selected rows, from the bf16 inputs, with no smoothing
+ * and no quantisation: O = softmax(q.K^T * sm_scale) . V over the kept keys (mask
+ * semantics as above; NULL = all keys).  out: fp64 [nrows, d]; a row with no kept key
+ * gives 0. */
+void sa_oracle_exact_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
+                          int H, int N, int d, double sm_scale, const uint8_t *mask,
+                          const int64_t *rows, int64_t nrows, double *out)
+{
+    (void)B; (void)H;
+    const int64_t nq = cdiv64(N, QBLK), nk = cdiv64(N, KBLK);
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    for (int64_t n = 0; n < nrows; ++n) {
+        const int64_t bh = rows[2 * n], r = rows[2 * n + 1];
+        const int64_t i = r / QBLK;
+        const uint16_t *qr = q + (bh * N + r) * d;
+        const uint16_t *kh = k + bh * N * d;
+        const uint16_t *vh = v + bh * N * d;
+        double mx = -INFINITY;
+        for (int64_t t = 0; t < N; ++t) {
+            int keep = !mask || mask[(bh * nq + i) * nk + t / KBLK];
+            if (!keep) { s[t] = -INFINITY; continue; }
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += (double)bf16_to_f32(qr[c]) * (double)bf16_to_f32(kh[t * d + c]);
+            s[t] = acc * sm_scale;
+            if (s[t] > mx) mx = s[t];
+        }
+        double *o = out + n * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (mx == -INFINITY) continue;
+        double den = 0.0;
+        for (int64_t t = 0; t < N; ++t) {
+            if (s[t] == -INFINITY) continue;
+            double p = exp(s[t] - mx);
+            den += p;
+            for (int c = 0; c < d; ++c) o[c] += p * (double)bf16_to_f32(vh[t * d + c]);
+        }
+        for (int c = 0; c < d; ++c) o[c] /= den;
+    }
+    free(s);
+}
+
+/* int32 S = q_i8 . k_i8^T for selected query rows against all Npad key rows (padded
+ * keys included, which are zero codes).  rows as above; out: int32 [nrows, Npad]. */
+void sa_oracle_qk_s32_rows(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
+                           const int64_t *rows, int64_t nrows, int32_t *out)
+{
+    (void)B; (void)H;
+    const int64_t Npad = padded_len(N);
+    for (int64_t n = 0; n < nrows; ++n) {
+        const int64_t bh = rows[2 * n], r = rows[2 * n + 1];
+        const int8_t *qr = q_i8 + (bh * Npad + r) * d;
+        const int8_t *kh = k_i8 + bh * Npad * d;
+        for (int64_t t = 0; t < Npad; ++t) {
+            int32_t S = 0;
+            for (int c = 0; c < d; ++c) S += (int32_t)qr[c] * (int32_t)kh[t * d + c];
+            out[n * Npad + t] = S;
+        }
+    }
+}
