@@ -1,0 +1,340 @@
+"""Benchmark of the low-bit attention forward (prologue + fused attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one sa_attn_fwd call over the whole workload (K mean, Q/K INT8 quantisation,
+V FP8 quantisation, fused INT8/FP8 attention), inputs resident in HBM.  Metric: tensor
+ops 4*B*H*N^2*d per second (the two contractions of dense attention).  Rank 0 prints one
+JSON line.  Under torchrun every rank runs its own replica of the workload (heads and
+batches are independent: no collective on the data path) and the reported time is the
+maximum over ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_attention_sa_b200.workloads import WORKLOADS, make_workload  # noqa: E402
+
+METRIC = "quantized attention TOPS (4·H·N²·d/s) and % of B200 dense INT8/FP8 peak"
+DEFAULT_WORKLOAD = "wan14b-720p-h40-n75600"
+DATASHEET_TOPS = 4500.0  # B200 dense INT8 / FP8 tensor peak (NVIDIA datasheet)
+KERNELS_PER_STEP = 6      # k_partial, k_mean, qk_quant, v_amax, v_quant, attn_fwd
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peak():
+    """8-bit tensor peak in TOPS from the measured bf16 cuBLAS burst figure times the
+    nominal 8-bit/bf16 ratio (4.5 / 2.25 PFLOP/s dense)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            m = json.load(f)
+        return 2.0 * float(m["bf16_tflops"]), "measured bf16 burst x 2 (nominal 8-bit/bf16 ratio)"
+    except Exception:
+        return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2 (nominal 8-bit/bf16 ratio)"
+
+
+def recorded_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    src = os.path.join(ROOT, "bit_quantized_attention_sa_b200", "csrc", "sa_attn.cu")
+    try:
+        with open(p) as f:
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()
+        if rec.get("sa_attn_cu_sha256") != h:
+            return None
+        return rec
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ CPU oracle arm
+
+
+def oracle_sample(w, q, k, v, m, rows_per_head: int):
+    """Times the CPU oracle on a bounded sample of the workload: the prologue of one head
+    and `rows_per_head` query rows of it.  Returns (ops_equiv, seconds, description)."""
+    import oracle
+    oracle.build()
+    h = 0
+    qh, kh, vh = (np.ascontiguousarray(x[:1, h:h + 1]) for x in (q, k, v))
+    mh = np.ascontiguousarray(m[:1, h:h + 1]) if m is not None else None
+    t0 = time.perf_counter()
+    qk = oracle.quantize_qk(qh, kh)
+    vq = oracle.quantize_v(vh)
+    t_pro = time.perf_counter() - t0
+    rng = np.random.default_rng(0)
+    rows = [(0, int(r)) for r in rng.choice(w.N, size=rows_per_head, replace=False)]
+    t0 = time.perf_counter()
+    oracle.attn_rows(qk, vq, w.N, w.sm_scale, rows, mh, 2)
+    t_rows = time.perf_counter() - t0
+    # the prologue serves all N rows of the head: charge the sampled rows their share
+    secs = t_rows + t_pro * rows_per_head / w.N
+    ops = 4.0 * rows_per_head * w.N * w.d
+    desc = (f"1 head of {w.name}: prologue ({t_pro:.2f} s, charged {rows_per_head}/{w.N}) + "
+            f"{rows_per_head} random query rows ({t_rows:.2f} s); single-threaded C oracle")
+    return ops, secs, desc
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    q, k, v, m = make_workload(w)
+    rows = args.oracle_rows
+    vals = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        ops, secs, desc = oracle_sample(w, q, k, v, m, rows)
+        if i >= args.warmup:
+            vals.append(ops / secs / 1e12)
+    value = float(np.median(vals)) if vals else 0.0
+    dense_step_s = w.dense_ops / (value * 1e12) if value > 0 else None
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dense_step_s * 1e3 if dense_step_s else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8+fp8e4m3 (emulated in fp32 on the CPU)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "mask_density": w.mask_density, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------ GPU arm
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--oracle-rows", type=int, default=48,
+                    help="query rows in the CPU oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=300))
+
+    from bit_quantized_attention_sa_b200 import binding as sa
+
+    # each rank owns one replica of the workload (its own seed)
+    q, k, v, m = make_workload(w) if rank == 0 else make_workload(
+        type(w)(w.name, w.B, w.H, w.N, w.d, w.outliers, w.mask_density, w.seed + 7919 * rank))
+    shape = (w.B, w.H, w.N, w.d)
+
+    def pinned_bf16(a):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory()
+
+    hq, hk, hv = pinned_bf16(q), pinned_bf16(k), pinned_bf16(v)
+    dq, dk, dv = (t.to(dev) for t in (hq, hk, hv))
+    dm = torch.from_numpy(m).to(dev) if m is not None else None
+    do = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def step():
+        sa.sa_attn_fwd(dq, dk, dv, w.sm_scale, block_mask=dm, out=do)
+
+    # ---- device-resident timing of the whole step
+    for _ in range(args.warmup):
+        step()
+    assert sa.sa_get_device_status() == 0
+    sampler = ClockSampler(local_rank)
+    barrier()
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    t_step = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.steps)
+    assert sa.sa_get_device_status() == 0
+
+    # ---- the attention kernel alone (dominant kernel): per-launch duration
+    q8, sq, k8, sk, _ = sa.sa_quantize_qk(dq, dk)
+    vt, sv = sa.sa_quantize_v(dv)
+    for _ in range(args.warmup):
+        sa.sa_attn_fwd_quantized(q8, sq, k8, sk, vt, sv, w.N, w.sm_scale, dm, out=do)
+    barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        sa.sa_attn_fwd_quantized(q8, sq, k8, sk, vt, sv, w.N, w.sm_scale, dm, out=do)
+    a1.record(stream)
+    barrier()
+    t_attn = max_over_ranks(a0.elapsed_time(a1) / 1e3 / args.steps)
+    del q8, k8, vt
+
+    # ---- end to end through the public API with host buffers
+    h2d = 3 * hq.numel() * 2
+    d2h = ho.numel() * 2
+    for _ in range(1):
+        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True); step(); ho.copy_(do, non_blocking=True)
+    barrier()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 5))
+    b0.record(stream)
+    for _ in range(e2e_steps):
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        step()
+        ho.copy_(do, non_blocking=True)
+    b1.record(stream)
+    barrier()
+    t_e2e = max_over_ranks(b0.elapsed_time(b1) / 1e3 / e2e_steps)
+
+    ops_rank = w.dense_ops
+    value = ops_rank * world / t_step / 1e12
+    peak, peak_src = measured_peak()
+    achieved = ops_rank / t_attn / 1e12
+    traffic = recorded_traffic()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ops_c, secs_c, desc = oracle_sample(w, q, k, v, m, args.oracle_rows)
+        cpu = {"value": ops_c / secs_c / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8+fp8e4m3", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                       "mask_density": w.mask_density, "sm_scale": w.sm_scale,
+                       "step": "sa_attn_fwd: K mean + Q/K INT8 + V FP8 prologue + fused attention",
+                       "l2": "inputs larger than L2 (each bf16 tensor %.0f MB)" % (h2d / 3 / 1e6),
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": peak_src,
+                         "frac_of_datasheet_4500": achieved / DATASHEET_TOPS,
+                         "ms_per_launch": t_attn * 1e3,
+                         "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
+            "cpu_baseline": cpu,
+            "e2e": {"value": ops_rank * world / t_e2e / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": t_e2e * 1e3},
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
+            "clocks": clocks,
+        }
+        if w.mask_density is not None and m is not None:
+            kept = int(m.sum())
+            exe = 4.0 * w.d * 128 * 64 * kept
+            line["config"]["mask_kept_fraction"] = kept / m.size
+            line["executed_tflops"] = exe / t_step / 1e12 * world
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

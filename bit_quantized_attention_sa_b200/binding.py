@@ -1,0 +1,209 @@
+"""Python binding of libsa.so: the C-ABI entry points of include/sa.h under the same
+names, taking torch tensors.  This module only marshals arguments (checks dtypes and
+shapes, allocates outputs with torch, passes raw pointers and the current CUDA stream);
+every step of the computation runs in the library's CUDA kernels.  There is no CPU
+fallback: importing this module raises if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libsa.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m bit_quantized_attention_sa_b200.build`"
+        " (there is no CPU fallback)")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+_lib.sa_quantize_qk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
+_lib.sa_quantize_v.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
+_lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
+_lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
+_lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
+_lib.sa_debug_wait_timeout.argtypes = [_I, _P]
+_lib.sa_get_device_status.argtypes = []
+_lib.sa_status_string.argtypes = [_I]
+_lib.sa_status_string.restype = ctypes.c_char_p
+_lib.sa_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.sa_workspace_bytes.restype = ctypes.c_size_t
+_lib.sa_release_workspace.argtypes = []
+_lib.sa_padded_len.argtypes = [_I]
+_lib.sa_padded_len.restype = ctypes.c_int64
+for _name in ("sa_quantize_qk", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_quantized",
+              "sa_debug_qk_s32", "sa_debug_wait_timeout", "sa_get_device_status",
+              "sa_release_workspace"):
+    getattr(_lib, _name).restype = _I
+
+SA_OK = 0
+STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED",
+                3: "SA_ERR_MISALIGNED", 4: "SA_ERR_CUDA", 5: "SA_ERR_OOM",
+                6: "SA_ERR_DEVICE_TIMEOUT"}
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {sa_status_string(status)} ({status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def raw_library() -> ctypes.CDLL:
+    """The ctypes handle itself (for tests of the C ABI)."""
+    return _lib
+
+
+def sa_status_string(status: int) -> str:
+    return _lib.sa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != SA_OK:
+        raise SAError(status, what)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dims(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, H, N, d] tensor")
+    B, H, N, d = q.shape
+    return int(B), int(H), int(N), int(d)
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str):
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def padded_len(N: int) -> int:
+    return int(_lib.sa_padded_len(int(N)))
+
+
+def sa_quantize_qk(q: torch.Tensor, k: torch.Tensor):
+    """Returns (q_i8 [B,H,Npad,d], q_scale [B,H,nq], k_i8 [B,H,Npad,d], k_scale [B,H,nk],
+    k_mean [B,H,d])."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    B, H, N, d = _dims(q)
+    if tuple(k.shape) != (B, H, N, d):
+        raise ValueError("q and k shapes differ")
+    Np, nq, nk = padded_len(N), -(-N // 128), -(-N // 64)
+    dev = q.device
+    q_i8 = torch.empty((B, H, Np, d), dtype=torch.int8, device=dev)
+    k_i8 = torch.empty((B, H, Np, d), dtype=torch.int8, device=dev)
+    q_scale = torch.empty((B, H, nq), dtype=torch.float32, device=dev)
+    k_scale = torch.empty((B, H, nk), dtype=torch.float32, device=dev)
+    k_mean = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    _check(_lib.sa_quantize_qk(_ptr(q), _ptr(k), B, H, N, d, _ptr(q_i8), _ptr(q_scale),
+                               _ptr(k_i8), _ptr(k_scale), _ptr(k_mean), _stream(dev)),
+           "sa_quantize_qk")
+    return q_i8, q_scale, k_i8, k_scale, k_mean
+
+
+def sa_quantize_v(v: torch.Tensor):
+    """Returns (v_fp8_t uint8 e4m3 [B,H,d,Npad], v_scale [B,H,d])."""
+    _need(v, torch.bfloat16, "v")
+    B, H, N, d = _dims(v)
+    Np = padded_len(N)
+    v_t = torch.empty((B, H, d, Np), dtype=torch.uint8, device=v.device)
+    v_scale = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
+    _check(_lib.sa_quantize_v(_ptr(v), B, H, N, d, _ptr(v_t), _ptr(v_scale), _stream(v.device)),
+           "sa_quantize_v")
+    return v_t, v_scale
+
+
+def _mask_arg(block_mask, B, H, N, device):
+    if block_mask is None:
+        return None
+    _need(block_mask, torch.uint8, "block_mask")
+    if tuple(block_mask.shape) != (B, H, -(-N // 128), -(-N // 64)) or block_mask.device != device:
+        raise ValueError("block_mask must be uint8 [B, H, ceil(N/128), ceil(N/64)] on q's device")
+    return block_mask
+
+
+def sa_attn_fwd(q, k, v, sm_scale: float | None = None, block_mask=None, out=None):
+    """bf16 [B,H,N,d] q, k, v -> bf16 O.  sm_scale defaults to 1/sqrt(d)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = _dims(q)
+    if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
+        raise ValueError("q, k, v shapes differ")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    m = _mask_arg(block_mask, B, H, N, q.device)
+    o = torch.empty_like(q) if out is None else out
+    _need(o, torch.bfloat16, "out")
+    _check(_lib.sa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, float(sm_scale),
+                            _ptr(m), _stream(q.device)), "sa_attn_fwd")
+    return o
+
+
+def sa_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v_fp8_t, v_scale, N: int,
+                          sm_scale: float | None = None, block_mask=None, out=None):
+    """The attention kernel on quantised inputs (layouts of sa_quantize_qk/v)."""
+    _need(q_i8, torch.int8, "q_i8")
+    _need(k_i8, torch.int8, "k_i8")
+    _need(v_fp8_t, torch.uint8, "v_fp8_t")
+    for t, n in ((q_scale, "q_scale"), (k_scale, "k_scale"), (v_scale, "v_scale")):
+        _need(t, torch.float32, n)
+    B, H, Np, d = _dims(q_i8)
+    if Np != padded_len(N):
+        raise ValueError("q_i8 is not padded to 128 * ceil(N/128) rows")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    m = _mask_arg(block_mask, B, H, N, q_i8.device)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q_i8.device) if out is None else out
+    _need(o, torch.bfloat16, "out")
+    _check(_lib.sa_attn_fwd_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale),
+                                      _ptr(v_fp8_t), _ptr(v_scale), _ptr(o), B, H, N, d,
+                                      float(sm_scale), _ptr(m), _stream(q_i8.device)),
+           "sa_attn_fwd_quantized")
+    return o
+
+
+def sa_debug_qk_s32(q_i8, k_i8, N: int):
+    """int32 S [B,H,Npad,Npad] from the tcgen05 INT8 path (small problems only)."""
+    _need(q_i8, torch.int8, "q_i8")
+    _need(k_i8, torch.int8, "k_i8")
+    B, H, Np, d = _dims(q_i8)
+    s = torch.empty((B, H, Np, Np), dtype=torch.int32, device=q_i8.device)
+    _check(_lib.sa_debug_qk_s32(_ptr(q_i8), _ptr(k_i8), B, H, N, d, _ptr(s),
+                                _stream(q_i8.device)), "sa_debug_qk_s32")
+    return s
+
+
+def sa_debug_wait_timeout(timeout_us: int, device=None):
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(_lib.sa_debug_wait_timeout(int(timeout_us), _stream(dev)), "sa_debug_wait_timeout")
+
+
+def sa_get_device_status() -> int:
+    """Synchronises the current device; returns and clears its device status word."""
+    return int(_lib.sa_get_device_status())
+
+
+def sa_workspace_bytes(B: int, H: int, N: int, d: int = 128) -> int:
+    return int(_lib.sa_workspace_bytes(B, H, N, d))
+
+
+def sa_release_workspace():
+    _check(_lib.sa_release_workspace(), "sa_release_workspace")

@@ -1,0 +1,342 @@
+// sa_api.cu -- the C ABI declared in include/sa.h: argument validation, the per-device
+// grow-only workspace, TMA tensor-map encoding and launch sequencing on the caller's
+// stream.  No entry point synchronises except sa_get_device_status and
+// sa_release_workspace.
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sa.h"
+#include "sa_internal.h"
+
+namespace sa {
+
+// ------------------------------------------------------------------ tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                       CUtensorMapSwizzle swizzle)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_stride_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ validation
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static sa_status check_shape(int B, int H, int N, int d, Shape *s)
+{
+    if (B < 1 || H < 1 || N < 1) return SA_ERR_INVALID_ARG;
+    if (d != kD) return SA_ERR_UNSUPPORTED;
+    s->B = B;
+    s->H = H;
+    s->N = N;
+    // TMA row coordinates and tile indices are 32-bit
+    if (s->BH() > INT_MAX / 8 || s->BH() * s->Npad() > INT_MAX) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+}
+
+static sa_status check_ptrs(std::initializer_list<const void *> ps)
+{
+    for (const void *p : ps)
+        if (!p) return SA_ERR_INVALID_ARG;
+    for (const void *p : ps)
+        if (!aligned16(p)) return SA_ERR_MISALIGNED;
+    return SA_OK;
+}
+
+// sm_100 device check, cached per device.
+static sa_status check_device()
+{
+    static int cached[64];  // 0 unknown, 1 ok, 2 unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? SA_OK : SA_ERR_UNSUPPORTED;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return SA_ERR_CUDA;
+    const bool ok = (major == 10 && minor == 0);
+    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    return ok ? SA_OK : SA_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------ workspace
+
+struct WsLayout {
+    size_t q8, k8, v8, sq, sk, sv, kmean, kpart, vamax, total;
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static WsLayout ws_layout(const Shape &s)
+{
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+    const size_t BH = size_t(s.BH()), Np = size_t(s.Npad());
+    L.q8 = take(BH * Np * kD);
+    L.k8 = take(BH * Np * kD);
+    L.v8 = take(BH * Np * kD);
+    L.sq = take(BH * size_t(s.nq()) * 4);
+    L.sk = take(BH * size_t(s.nk()) * 4);
+    L.sv = take(BH * kD * 4);
+    L.kmean = take(BH * kD * 4);
+    L.kpart = take(BH * size_t(s.nchunks()) * kD * 8);
+    L.vamax = take(BH * kD * 4);
+    L.total = off;
+    return L;
+}
+
+struct DeviceWs {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+static DeviceWs g_ws[64];
+static std::mutex g_ws_mutex;
+
+// Returns the current device's workspace grown to at least `bytes`.
+static sa_status get_workspace(size_t bytes, uint8_t **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    DeviceWs &w = g_ws[dev];
+    if (w.bytes < bytes) {
+        if (w.ptr) {
+            // earlier work on any stream may still use the old buffer
+            if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;
+            cudaFree(w.ptr);
+            w.ptr = nullptr;
+            w.bytes = 0;
+        }
+        if (cudaMalloc(&w.ptr, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            w.ptr = nullptr;
+            return SA_ERR_OOM;
+        }
+        w.bytes = bytes;
+    }
+    *out = static_cast<uint8_t *>(w.ptr);
+    return SA_OK;
+}
+
+static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t *k8,
+                                const float *sk, const uint8_t *v8, const float *sv, void *o,
+                                const Shape &s, float sm_scale, const uint8_t *mask,
+                                cudaStream_t st)
+{
+    AttnArgs a;
+    const uint64_t rows = uint64_t(s.BH() * s.Npad());
+    if (!encode_tmap_2d_u8(&a.tm_q, q8, kD, rows, kD, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d_u8(&a.tm_k, k8, kD, rows, kD, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d_u8(&a.tm_v, v8, uint64_t(s.Npad()), uint64_t(s.BH()) * kD,
+                           uint64_t(s.Npad()), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+        return SA_ERR_CUDA;
+    a.q_scale = sq;
+    a.k_scale = sk;
+    a.v_scale = sv;
+    a.mask = mask;
+    a.o = static_cast<__nv_bfloat16 *>(o);
+    a.BH = int(s.BH());
+    a.N = int(s.N);
+    a.Npad = int(s.Npad());
+    a.nq = int(s.nq());
+    a.nk = int(s.nk());
+    a.sm_scale = sm_scale;
+    return launch_attention(a, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+sa_status sa_quantize_qk(const void *q, const void *k, int B, int H, int N, int d,
+                         int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                         float *k_mean, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({q, k, q_i8, q_scale, k_i8, k_scale, k_mean})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    const WsLayout L = ws_layout(s);
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(L.total, &ws)) != SA_OK) return r;
+    cudaError_t e = launch_quantize_qk(q, k, s, q_i8, q_scale, k_i8, k_scale, k_mean,
+                                       reinterpret_cast<double *>(ws + L.kpart),
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp8_t,
+                        float *v_scale, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({v, v_fp8_t, v_scale})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    const WsLayout L = ws_layout(s);
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(L.total, &ws)) != SA_OK) return r;
+    cudaError_t e = launch_quantize_v(v, s, v_fp8_t, v_scale,
+                                      reinterpret_cast<uint32_t *>(ws + L.vamax),
+                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                      int N, int d, float sm_scale, const uint8_t *block_mask, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
+    if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    const WsLayout L = ws_layout(s);
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(L.total, &ws)) != SA_OK) return r;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int8_t *q8 = reinterpret_cast<int8_t *>(ws + L.q8);
+    int8_t *k8 = reinterpret_cast<int8_t *>(ws + L.k8);
+    uint8_t *v8 = ws + L.v8;
+    float *sq = reinterpret_cast<float *>(ws + L.sq);
+    float *sk = reinterpret_cast<float *>(ws + L.sk);
+    float *sv = reinterpret_cast<float *>(ws + L.sv);
+    if (launch_quantize_qk(q, k, s, q8, sq, k8, sk, reinterpret_cast<float *>(ws + L.kmean),
+                           reinterpret_cast<double *>(ws + L.kpart), st) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st) !=
+        cudaSuccess)
+        return SA_ERR_CUDA;
+    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st);
+}
+
+sa_status sa_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                                const float *k_scale, const uint8_t *v_fp8_t,
+                                const float *v_scale, void *o, int B, int H, int N, int d,
+                                float sm_scale, const uint8_t *block_mask, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
+    if ((r = check_ptrs({q_i8, k_i8, v_fp8_t, o})) != SA_OK) return r;
+    if (!q_scale || !k_scale || !v_scale) return SA_ERR_INVALID_ARG;
+    if ((r = check_device()) != SA_OK) return r;
+    return attention_core(q_i8, q_scale, k_i8, k_scale, v_fp8_t, v_scale, o, s, sm_scale,
+                          block_mask, static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
+                          int32_t *s_out, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({q_i8, k_i8, s_out})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    CUtensorMap tq, tk;
+    const uint64_t rows = uint64_t(s.BH() * s.Npad());
+    if (!encode_tmap_2d_u8(&tq, q_i8, kD, rows, kD, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d_u8(&tk, k_i8, kD, rows, kD, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return SA_ERR_CUDA;
+    return launch_debug_qk_s32(tq, tk, int(s.BH()), int(s.Npad()), s_out,
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+sa_status sa_debug_wait_timeout(int timeout_us, void *stream)
+{
+    if (timeout_us < 1 || timeout_us > 10000000) return SA_ERR_INVALID_ARG;
+    sa_status r = check_device();
+    if (r != SA_OK) return r;
+    return launch_debug_wait_timeout(timeout_us, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+sa_status sa_get_device_status(void)
+{
+    int st = 0;
+    if (read_and_clear_status(&st) != cudaSuccess) return SA_ERR_CUDA;
+    return st == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
+}
+
+const char *sa_status_string(sa_status s)
+{
+    switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_MISALIGNED: return "SA_ERR_MISALIGNED";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_OOM: return "SA_ERR_OOM";
+    case SA_ERR_DEVICE_TIMEOUT: return "SA_ERR_DEVICE_TIMEOUT";
+    }
+    return "SA_ERR_UNKNOWN";
+}
+
+size_t sa_workspace_bytes(int B, int H, int N, int d)
+{
+    Shape s;
+    if (check_shape(B, H, N, d, &s) != SA_OK) return 0;
+    return ws_layout(s).total;
+}
+
+sa_status sa_release_workspace(void)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    DeviceWs &w = g_ws[dev];
+    if (w.ptr) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;
+        cudaFree(w.ptr);
+        w.ptr = nullptr;
+        w.bytes = 0;
+    }
+    return SA_OK;
+}
+
+int64_t sa_padded_len(int N) { return N < 1 ? 0 : sa::padded_len(N); }
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// sa_internal.h -- launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace sa {
+
+constexpr int kD = 128;      // head dimension
+constexpr int kQBlk = 128;   // query tokens per quantisation block / tile / mask row
+constexpr int kKBlk = 64;    // key tokens per quantisation block / mask column
+constexpr int kMeanChunk = 1024;  // tokens per partial-sum block of the K mean
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t padded_len(int64_t n) { return cdiv(n, kQBlk) * kQBlk; }
+
+struct Shape {
+    int64_t B, H, N;
+    int64_t BH() const { return B * H; }
+    int64_t Npad() const { return padded_len(N); }
+    int64_t nq() const { return cdiv(N, kQBlk); }
+    int64_t nk() const { return cdiv(N, kKBlk); }
+    int64_t nchunks() const { return cdiv(N, kMeanChunk); }
+};
+
+// ---- prologue (sa_prologue.cu)
+cudaError_t launch_quantize_qk(const void *q, const void *k, const Shape &s, int8_t *q_i8,
+                               float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
+                               double *k_partial /* [BH, nchunks, d] */, cudaStream_t st);
+cudaError_t launch_quantize_v(const void *v, const Shape &s, uint8_t *v_t, float *v_scale,
+                              uint32_t *v_amax_bits /* [BH, d] */, cudaStream_t st);
+
+// ---- attention (sa_attn.cu)
+struct AttnArgs {
+    CUtensorMap tm_q, tm_k, tm_v;
+    const float *q_scale, *k_scale, *v_scale;
+    const uint8_t *mask;
+    __nv_bfloat16 *o;
+    int BH, N, Npad, nq, nk;
+    float sm_scale;
+};
+cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
+cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k, int BH,
+                                int Npad, int32_t *s_out, cudaStream_t st);
+cudaError_t launch_debug_wait_timeout(int timeout_us, cudaStream_t st);
+// Reads and clears the device status word of the current device (synchronous).
+cudaError_t read_and_clear_status(int *status);
+
+// ---- tensor maps (sa_api.cu)
+bool encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                       uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                       CUtensorMapSwizzle swizzle);
+
+}  // namespace sa

@@ -1,0 +1,290 @@
+// sa_prologue.cu -- the quantise/smooth prologue: K channel means, INT8 Q and smoothed K
+// per block, FP8 e4m3 V per channel written channel-major.  All passes are HBM-bound
+// streams over [B,H,N,128] bf16 tensors; each thread moves 16-byte chunks (8 channels of
+// one token) so every warp access is a fully used 256-byte row pair.
+//
+// Sources: "AIGC weekend special 5.10", section 1.2 Method item (1) (Q/K to INT8 for the
+// tensor cores); "Video-Generation-101: inference systems" reference [3] (outlier
+// smoothing, read as subtracting K's per-channel token mean); "Video-Generation-101
+// research log" section 5.5 (FP8 P.V, so V in FP8).
+//
+// Bit-exactness: scales are IEEE fp32 divisions amax/127 and amax/448, codes use IEEE
+// division followed by round-to-nearest-even (cvt.rni) or the e4m3 round-to-nearest-even
+// saturating conversion.  This file must not be built with fast-math or -prec-div=false.
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sa_internal.h"
+#include "sa_ptx.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8])
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = bf16_bits_to_f32(w[i] & 0xFFFFu);
+        x[2 * i + 1] = bf16_bits_to_f32(w[i] >> 16);
+    }
+}
+
+// ---- K channel sums: per (head, 1024-token chunk) fp64 partial sums, fixed order.
+__global__ void __launch_bounds__(kThreads) k_partial_kernel(const uint16_t *__restrict__ k,
+                                                             int N, int nchunks,
+                                                             double *__restrict__ part)
+{
+    __shared__ double red[16][kD];
+    const int chunk = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
+    const int t0 = chunk * kMeanChunk;
+    const int t1 = min(N, t0 + kMeanChunk);
+    const uint16_t *kh = k + bh * int64_t(N) * kD;
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+    for (int t = t0 + rs; t < t1; t += 16) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(kh + int64_t(t) * kD + cg * 8));
+        float x[8];
+        unpack8(u, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += double(x[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rs][cg * 8 + e] = acc[e];
+    __syncthreads();
+    if (tid < kD) {
+        double s = 0.0;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) s += red[r][tid];
+        part[(bh * nchunks + chunk) * kD + tid] = s;
+    }
+}
+
+// mean_k[c] = fp32( (sum over chunks, in order) / N ) in fp64.
+__global__ void __launch_bounds__(kD) k_mean_kernel(const double *__restrict__ part, int N,
+                                                    int nchunks, float *__restrict__ mean)
+{
+    const int64_t bh = blockIdx.x;
+    const int c = threadIdx.x;
+    double s = 0.0;
+    for (int i = 0; i < nchunks; ++i) s += part[(bh * nchunks + i) * kD + c];
+    mean[bh * kD + c] = float(s / double(N));
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ int8_t int8_code(float x, float s)
+{
+    if (s == 0.0f) return 0;
+    int r = __float2int_rn(__fdiv_rn(x, s));
+    r = max(-127, min(127, r));
+    return int8_t(r);
+}
+
+// One quantisation block of ROWS tokens x 128 channels starting at token r0.
+// mean != nullptr: smooth first (x - mean[c], one fp32 subtraction).  Rows >= N are
+// excluded from the max and stored as zero codes.  scale_out may be null (padding-only
+// block).
+template <int ROWS>
+__device__ __forceinline__ void quant_block(const uint16_t *__restrict__ src, int N, int r0,
+                                            const float *__restrict__ mean,
+                                            int8_t *__restrict__ dst, float *scale_out,
+                                            float *red)
+{
+    constexpr int PER = ROWS * 16 / kThreads;  // 16-byte chunks per thread
+    const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
+    float x[PER][8];
+    float mc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mc[e] = mean ? mean[cg * 8 + e] : 0.0f;
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int t = r0 + rs + 16 * i;
+        if (t < N) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + int64_t(t) * kD + cg * 8));
+            unpack8(u, x[i]);
+            if (mean) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) x[i][e] = __fsub_rn(x[i][e], mc[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[i][e] = 0.0f;
+        }
+    }
+    amax = warp_max(amax);
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    amax = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+    const float s = __fdiv_rn(amax, 127.0f);
+    if (tid == 0 && scale_out) *scale_out = s;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int t = r0 + rs + 16 * i;
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) lo |= uint32_t(uint8_t(int8_code(x[i][e], s))) << (8 * e);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hi |= uint32_t(uint8_t(int8_code(x[i][4 + e], s))) << (8 * e);
+        *reinterpret_cast<uint2 *>(dst + int64_t(t) * kD + cg * 8) = make_uint2(lo, hi);
+    }
+}
+
+// grid (nq + Npad/64, BH): x < nq quantises Q block x; otherwise K block x - nq
+// (blocks at or past nk only zero-fill the padded key rows).
+__global__ void __launch_bounds__(kThreads)
+    qk_quant_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, int N,
+                    int Npad, int nq, int nk, const float *__restrict__ kmean,
+                    int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
+                    int8_t *__restrict__ k_i8, float *__restrict__ k_scale)
+{
+    __shared__ float red[kThreads / 32];
+    const int64_t bh = blockIdx.y;
+    const int x = blockIdx.x;
+    if (x < nq) {
+        quant_block<kQBlk>(q + bh * int64_t(N) * kD, N, x * kQBlk, nullptr,
+                           q_i8 + bh * int64_t(Npad) * kD, q_scale + bh * nq + x, red);
+    } else {
+        const int j = x - nq;
+        quant_block<kKBlk>(k + bh * int64_t(N) * kD, N, j * kKBlk, kmean + bh * kD,
+                           k_i8 + bh * int64_t(Npad) * kD, j < nk ? k_scale + bh * nk + j : nullptr,
+                           red);
+    }
+}
+
+// ---- V: per-channel max |v| (as bf16 magnitude bits; order-free), then codes.
+__global__ void __launch_bounds__(kThreads) v_amax_kernel(const uint16_t *__restrict__ v, int N,
+                                                          uint32_t *__restrict__ amax_bits)
+{
+    __shared__ uint32_t red[16][kD];
+    const int chunk = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
+    const int t0 = chunk * kMeanChunk;
+    const int t1 = min(N, t0 + kMeanChunk);
+    const uint16_t *vh = v + bh * int64_t(N) * kD;
+    uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int t = t0 + rs; t < t1; t += 16) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vh + int64_t(t) * kD + cg * 8));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            m[2 * i] = max(m[2 * i], w[i] & 0x7FFFu);
+            m[2 * i + 1] = max(m[2 * i + 1], (w[i] >> 16) & 0x7FFFu);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rs][cg * 8 + e] = m[e];
+    __syncthreads();
+    if (tid < kD) {
+        uint32_t r = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r = max(r, red[i][tid]);
+        atomicMax(amax_bits + bh * kD + tid, r);
+    }
+}
+
+// grid (Npad/128, BH): a 128-token x 128-channel tile, quantised and transposed through
+// shared memory so that both the bf16 reads and the channel-major FP8 writes are
+// coalesced 16-byte accesses.
+__global__ void __launch_bounds__(kThreads)
+    v_quant_kernel(const uint16_t *__restrict__ v, int N, int Npad,
+                   const uint32_t *__restrict__ amax_bits, uint8_t *__restrict__ v_t,
+                   float *__restrict__ v_scale)
+{
+    constexpr int kPitch = 144;  // bytes per channel row in shared memory (16-B multiple)
+    __shared__ __align__(16) uint8_t tile[kD][kPitch];
+    __shared__ float sv[kD];
+    const int64_t bh = blockIdx.y;
+    const int t0 = blockIdx.x * kQBlk;
+    const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
+    if (tid < kD) {
+        const float s = __fdiv_rn(bf16_bits_to_f32(amax_bits[bh * kD + tid]), 448.0f);
+        sv[tid] = s;
+        if (blockIdx.x == 0) v_scale[bh * kD + tid] = s;
+    }
+    __syncthreads();
+    const uint16_t *vh = v + bh * int64_t(N) * kD;
+#pragma unroll
+    for (int i = 0; i < kQBlk * 16 / kThreads; ++i) {
+        const int r = rs + 16 * i;
+        const int t = t0 + r;
+        float x[8];
+        if (t < N) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vh + int64_t(t) * kD + cg * 8));
+            unpack8(u, x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const float s0 = sv[cg * 8 + e], s1 = sv[cg * 8 + e + 1];
+            const float y0 = s0 == 0.0f ? 0.0f : __fdiv_rn(x[e], s0);
+            const float y1 = s1 == 0.0f ? 0.0f : __fdiv_rn(x[e + 1], s1);
+            const uint32_t p = pack_e4m3x2(y0, y1);
+            tile[cg * 8 + e][r] = uint8_t(p & 0xFFu);
+            tile[cg * 8 + e + 1][r] = uint8_t(p >> 8);
+        }
+    }
+    __syncthreads();
+    uint8_t *vt = v_t + bh * int64_t(kD) * Npad;
+#pragma unroll
+    for (int i = 0; i < kD * 8 / kThreads; ++i) {
+        const int qd = tid + kThreads * i;
+        const int c = qd >> 3, part = qd & 7;
+        const uint4 u = *reinterpret_cast<const uint4 *>(&tile[c][part * 16]);
+        *reinterpret_cast<uint4 *>(vt + int64_t(c) * Npad + t0 + part * 16) = u;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_qk(const void *q, const void *k, const Shape &s, int8_t *q_i8,
+                               float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
+                               double *k_partial, cudaStream_t st)
+{
+    const int N = int(s.N), Npad = int(s.Npad()), nq = int(s.nq()), nk = int(s.nk());
+    const int nch = int(s.nchunks());
+    const dim3 g1(nch, unsigned(s.BH()));
+    k_partial_kernel<<<g1, kThreads, 0, st>>>(static_cast<const uint16_t *>(k), N, nch, k_partial);
+    k_mean_kernel<<<unsigned(s.BH()), kD, 0, st>>>(k_partial, N, nch, k_mean);
+    const dim3 g2(nq + Npad / kKBlk, unsigned(s.BH()));
+    qk_quant_kernel<<<g2, kThreads, 0, st>>>(static_cast<const uint16_t *>(q),
+                                             static_cast<const uint16_t *>(k), N, Npad, nq, nk,
+                                             k_mean, q_i8, q_scale, k_i8, k_scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_v(const void *v, const Shape &s, uint8_t *v_t, float *v_scale,
+                              uint32_t *v_amax_bits, cudaStream_t st)
+{
+    const int N = int(s.N), Npad = int(s.Npad());
+    cudaError_t e = cudaMemsetAsync(v_amax_bits, 0, sizeof(uint32_t) * s.BH() * kD, st);
+    if (e != cudaSuccess) return e;
+    const dim3 g1(unsigned(s.nchunks()), unsigned(s.BH()));
+    v_amax_kernel<<<g1, kThreads, 0, st>>>(static_cast<const uint16_t *>(v), N, v_amax_bits);
+    const dim3 g2(unsigned(Npad / kQBlk), unsigned(s.BH()));
+    v_quant_kernel<<<g2, kThreads, 0, st>>>(static_cast<const uint16_t *>(v), N, Npad, v_amax_bits,
+                                            v_t, v_scale);
+    return cudaGetLastError();
+}
+
+}  // namespace sa

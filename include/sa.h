@@ -1,0 +1,133 @@
+/*
+ * sa.h -- C ABI of libsa.so, a B200 (sm_100a) SageAttention-style low-bit attention
+ * forward with optional SLA-style block sparsity.
+ *
+ * The method (sources, by page and section):
+ *   - "AIGC weekend special 5.10: full-stack optimisation of visual-generation
+ *     inference", section 1 (TurboDiffusion), 1.2 Method, item (1): SageAttention2++
+ *     quantises Q and K to low bit and runs Q.K^T on tensor cores; item (2): SLA
+ *     sparse attention is orthogonal to it and runs on top of it.
+ *   - "Video-Generation-101: inference systems", kernel paragraph and reference [3]:
+ *     format / thread-granularity / accumulation co-design with outlier smoothing.
+ *   - "Video-Generation-101 research log", section 5.5 table: INT4/INT8 Q.K^T with
+ *     FP8/FP16 P.V.
+ *   - NetEase article on the TurboDiffusion release, "attention acceleration" section
+ *     and the SLA figure caption: only the critical blocks of the attention weights
+ *     get exact (sparse) attention.
+ * Numerical definition implemented (the pages give the outline; each detail they leave
+ * open is stated here):
+ *   per (b,h): mean_k[c] = fp32( sum_t K[t,c] (fp64) / N );
+ *   Q: per 128-token block, scale_q = max|q| / 127, q_i8 = rint_even(q / scale_q);
+ *   K: ks = K - mean_k (fp32), per 64-token block scale_k = max|ks| / 127,
+ *      k_i8 = rint_even(ks / scale_k); codes clamp to [-127, 127]; zero block -> scale 0;
+ *   V: per channel scale_v = max_t |v| / 448, v_fp8 = e4m3_rn_satfinite(v / scale_v);
+ *   S = q_i8 . k_i8^T exact in int32; s = S * (scale_q * scale_k * sm_scale);
+ *   online softmax in fp32 over the kept 64-key blocks, two blocks per step;
+ *   p8 = e4m3(448 * exp(s - m)); l = sum of p8; acc = sum p8 * v_fp8 (fp32);
+ *   O = acc * scale_v / l (bf16), 0 for a row with no kept key.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are contiguous row-major.  q, k, v, o: bf16 [B,H,N,d].  d must be 128.
+ *     Npad = 128 * ceil(N/128); nq = ceil(N/128); nk = ceil(N/64).
+ *   - Device pointers are owned by the caller; the library never frees them.  All
+ *     pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
+ *     call only enqueues work on that stream and returns without synchronising, except
+ *     sa_get_device_status, which synchronises the device.
+ *   - Argument errors are detected on the host before any launch; outputs are then
+ *     untouched.  Launch failures return SA_ERR_CUDA.  Device-side bounded waits that
+ *     expire set a device status word read by sa_get_device_status.
+ *   - Block mask: uint8 [B,H,nq,nk], nonzero keeps the (128-query x 64-key) block; NULL
+ *     keeps every block.  Masked blocks are neither loaded nor computed.
+ */
+#ifndef SA_H
+#define SA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, size overflow */
+    SA_ERR_UNSUPPORTED = 2,    /* d != 128, or no sm_100 device */
+    SA_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
+    SA_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
+    SA_ERR_OOM = 5,            /* the library workspace could not be allocated */
+    SA_ERR_DEVICE_TIMEOUT = 6  /* a device-side bounded wait expired */
+} sa_status;
+
+/* Quantise Q and smooth + quantise K (the Q/K half of the prologue).
+ * Sources: TurboDiffusion digest 1.2(1) (Q/K to INT8 on tensor cores);
+ * Video-Generation-101 reference [3] (outlier smoothing).
+ * Outputs (device, caller-owned):
+ *   q_i8 int8 [B,H,Npad,d] (rows >= N zero), q_scale fp32 [B,H,nq],
+ *   k_i8 int8 [B,H,Npad,d] (rows >= N zero), k_scale fp32 [B,H,nk],
+ *   k_mean fp32 [B,H,d].
+ * Results are bit-identical to the definition above (the K mean whenever the fp64 sum
+ * of the column is exact, which holds for bf16 inputs of ordinary range).
+ * Uses the library workspace for per-block fp64 partial sums of K. */
+sa_status sa_quantize_qk(const void *q, const void *k, int B, int H, int N, int d,
+                         int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                         float *k_mean, void *stream);
+
+/* Quantise V to FP8 e4m3 per channel, stored transposed (the V half of the prologue).
+ * Source: Video-Generation-101 research log 5.5 (FP8 P.V).
+ * Outputs: v_fp8_t uint8 e4m3 [B,H,d,Npad] (keys contiguous, keys >= N zero),
+ *          v_scale fp32 [B,H,d].  Bit-identical to the definition above.
+ * Uses the library workspace for per-channel maxima. */
+sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp8_t,
+                        float *v_scale, void *stream);
+
+/* Full forward: prologue into the library workspace, then the fused attention kernel.
+ * Sources: all of the above; FlashAttention tiling (digest timeline, 2022.06) for the
+ * online softmax.  o: bf16 [B,H,N,d] (device, caller-owned).  sm_scale: the logit scale,
+ * normally 1/sqrt(d).  block_mask: see conventions, or NULL.
+ * The workspace is library-owned, per device, grow-only (cudaMalloc on first use or
+ * growth, so the first call at a new size must not be inside a stream capture). */
+sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
+                      int N, int d, float sm_scale, const uint8_t *block_mask, void *stream);
+
+/* The fused attention kernel alone, on already-quantised inputs (the layouts written by
+ * sa_quantize_qk and sa_quantize_v).  For callers that reuse quantised K/V across
+ * queries, and for timing the kernel without the prologue.  Allocates nothing. */
+sa_status sa_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                                const float *k_scale, const uint8_t *v_fp8_t,
+                                const float *v_scale, void *o, int B, int H, int N, int d,
+                                float sm_scale, const uint8_t *block_mask, void *stream);
+
+/* Debug: the int32 S = q_i8 . k_i8^T tiles computed by the same tcgen05 INT8 path the
+ * attention kernel uses, stored to s_out int32 [B,H,Npad,Npad] (padded rows/keys
+ * included).  For bit-exact checks on small problems only.  Allocates nothing. */
+sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
+                          int32_t *s_out, void *stream);
+
+/* Debug: launches a one-CTA kernel whose mbarrier wait can never complete, bounded by
+ * timeout_us microseconds; the kernel then records SA_ERR_DEVICE_TIMEOUT in the device
+ * status word and returns.  Exercises the failure path without faulting the GPU. */
+sa_status sa_debug_wait_timeout(int timeout_us, void *stream);
+
+/* Synchronises the current device, returns and clears its device status word
+ * (SA_OK or SA_ERR_DEVICE_TIMEOUT), or SA_ERR_CUDA if synchronisation failed. */
+sa_status sa_get_device_status(void);
+
+/* Human-readable name of a status code (static string). */
+const char *sa_status_string(sa_status s);
+
+/* Bytes of library workspace sa_attn_fwd needs for this problem size (0 on bad sizes). */
+size_t sa_workspace_bytes(int B, int H, int N, int d);
+
+/* Frees the current device's workspace (synchronises the device first). */
+sa_status sa_release_workspace(void);
+
+/* Padded token count Npad = 128 * ceil(N/128) (0 for N < 1). */
+int64_t sa_padded_len(int N);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H */

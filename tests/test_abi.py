@@ -1,0 +1,62 @@
+"""The C ABI without a GPU: the library loads, exports every entry point include/sa.h
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    text = open(os.path.join(ROOT, "include", "sa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(libsa):
+    names = declared_entry_points()
+    assert len(names) >= 10
+    lib = libsa.raw_library()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings_and_sizes(libsa):
+    assert libsa.sa_status_string(0) == "SA_OK"
+    assert libsa.sa_status_string(6) == "SA_ERR_DEVICE_TIMEOUT"
+    assert [libsa.padded_len(n) for n in (0, 1, 128, 129, 75600)] == [0, 128, 128, 256, 75648]
+    assert libsa.sa_workspace_bytes(1, 2, 1024, 64) == 0
+    assert libsa.sa_workspace_bytes(1, 2, 0, 128) == 0
+    ws = libsa.sa_workspace_bytes(1, 40, 75600, 128)
+    assert 3 * 40 * 75648 * 128 <= ws < 3 * 40 * 75648 * 128 + (1 << 24)
+
+
+FAKE = ctypes.c_void_p(1 << 20)       # 16-byte aligned, never dereferenced
+ODD = ctypes.c_void_p((1 << 20) + 8)  # misaligned
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0.088, None, None), 1),   # null q
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.088, None, None), 2),    # d != 128
+    ((FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, 0.088, None, None), 3),    # misaligned o
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 0.088, None, None), 1),     # N = 0
+    ((FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, 0.088, None, None), 1),   # B = 0
+    ((FAKE, FAKE, FAKE, FAKE, 1 << 20, 1 << 10, 128, 128, 0.088, None, None), 1),  # overflow
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0.0, None, None), 1),     # sm_scale <= 0
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, float("nan"), None, None), 1),
+])
+def test_attn_fwd_argument_errors(libsa, args, expect):
+    assert libsa.raw_library().sa_attn_fwd(*args) == expect
+
+
+def test_other_entry_points_argument_errors(libsa):
+    lib = libsa.raw_library()
+    assert lib.sa_quantize_qk(FAKE, None, 1, 1, 128, 128, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert lib.sa_quantize_qk(FAKE, FAKE, 1, 1, 128, 96, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert lib.sa_quantize_v(FAKE, 1, 1, 128, 128, ODD, FAKE, None) == 3
+    assert lib.sa_attn_fwd_quantized(FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 1, 128, 128,
+                                     ctypes.c_float(0.088), None, None) == 1
+    assert lib.sa_debug_qk_s32(FAKE, FAKE, 1, 1, -5, 128, FAKE, None) == 1
+    assert lib.sa_debug_wait_timeout(0, None) == 1
