@@ -31,6 +31,7 @@ _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
 _lib.sa_debug_wait_timeout.argtypes = [_I, _P]
+_lib.sa_debug_exp2_poly.argtypes = [_P, _P, _I, _P]
 _lib.sa_get_device_status.argtypes = []
 _lib.sa_status_string.argtypes = [_I]
 _lib.sa_status_string.restype = ctypes.c_char_p
@@ -40,7 +41,7 @@ _lib.sa_release_workspace.argtypes = []
 _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_quantized",
-              "sa_debug_qk_s32", "sa_debug_wait_timeout", "sa_get_device_status",
+              "sa_debug_qk_s32", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
 
@@ -194,6 +195,15 @@ def sa_debug_qk_s32(q_i8, k_i8, N: int):
 def sa_debug_wait_timeout(timeout_us: int, device=None):
     dev = torch.device("cuda") if device is None else torch.device(device)
     _check(_lib.sa_debug_wait_timeout(int(timeout_us), _stream(dev)), "sa_debug_wait_timeout")
+
+
+def sa_debug_exp2_poly(x: torch.Tensor) -> torch.Tensor:
+    """2^x by the attention kernel's polynomial exponential (fp32 CUDA tensor)."""
+    _need(x, torch.float32, "x")
+    y = torch.empty_like(x)
+    _check(_lib.sa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(x.device)),
+           "sa_debug_exp2_poly")
+    return y
 
 
 def sa_get_device_status() -> int:

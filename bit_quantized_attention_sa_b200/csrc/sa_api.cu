@@ -294,6 +294,17 @@ sa_status sa_debug_wait_timeout(int timeout_us, void *stream)
                : SA_ERR_CUDA;
 }
 
+sa_status sa_debug_exp2_poly(const float *x, float *y, int n, void *stream)
+{
+    if (n < 1) return SA_ERR_INVALID_ARG;
+    sa_status r = check_ptrs({x, y});
+    if (r != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    return launch_debug_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
 sa_status sa_get_device_status(void)
 {
     int st = 0;

@@ -75,6 +75,12 @@ static_assert(kVHalfBytes % 1024 == 0, "V half tiles stay 1024-B aligned");
 constexpr uint32_t kIdescQK = idesc_s8_s32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, kOCols);
 
+// Of every 4 softmax exponentials, this many run as a polynomial on the FMA/ALU pipes
+// (exp2_poly) instead of the MUFU pipe, to balance the two.
+#ifndef SA_POLY_OF_4
+#define SA_POLY_OF_4 1
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;
 
@@ -307,31 +313,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 const int2 jp = info[st];
                 const int j = ok ? (wg ? jp.y : jp.x) : -1;  // info is only valid once loaded
-                uint32_t sa[32], sbv[32];
-                if (ok && j >= 0) {
-                    tc_fence_after();
-                    const uint32_t taddr = tmem + lane_addr + (sb ? kColS1 : kColS0) + 64 * wg;
-                    tmem_ld32_wait(taddr, sa);
-                    tmem_ld32_wait(taddr + 32, sbv);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
+                const int nvalid = j >= 0 ? min(64, N - 64 * j) : 0;
+                const uint32_t taddr = tmem + lane_addr + (sb ? kColS1 : kColS0) + 64 * wg;
 
-                int nvalid = 0;
+                // pass 1: row max of this half, on int32 S (the scale is positive)
                 float c = 0.0f, pmax = -INFINITY;
                 if (j >= 0) {
-                    nvalid = min(64, N - 64 * j);
                     c = (sq * k_scale[int64_t(bh) * nk + j]) * sm_scale;
-                    int imax = INT_MIN;
+                    tc_fence_after();
+                    uint32_t a[32], b[32];
+                    tmem_ld64_wait(taddr, a, b);
+                    int imax;
                     if (nvalid == 64) {
+                        int acc[8];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) imax = max(imax, max(int(sa[i]), int(sbv[i])));
+                        for (int k = 0; k < 8; ++k) acc[k] = max(int(a[k]), int(b[k]));
+#pragma unroll
+                        for (int i = 8; i < 32; i += 8)
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) acc[k] = max(acc[k], max(int(a[i + k]), int(b[i + k])));
+                        imax = max(max(max(acc[0], acc[1]), max(acc[2], acc[3])),
+                                   max(max(acc[4], acc[5]), max(acc[6], acc[7])));
                     } else {
+                        imax = INT_MIN;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            if (i < nvalid) imax = max(imax, int(sa[i]));
-                            if (i + 32 < nvalid) imax = max(imax, int(sbv[i]));
+                            if (i < nvalid) imax = max(imax, int(a[i]));
+                            if (i + 32 < nvalid) imax = max(imax, int(b[i]));
                         }
                     }
                     pmax = i2f(uint32_t(imax)) * c;
@@ -342,38 +350,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float other = x[(wg ^ 1) * 128 + row];
                 const float mnew = fmaxf(m, fmaxf(pmax, other));
 
-                // P = e4m3(448 * exp(s - mnew)) for this half, 64 keys -> 16 words
-                uint32_t pw[16];
-                if (j >= 0) {
-                    const float c2 = c * kLog2e;
-                    const float nb = kLog2_448 - mnew * kLog2e;
-#pragma unroll
-                    for (int w = 0; w < 16; ++w) {
-                        float p[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int i = 4 * w + e;
-                            const uint32_t sij = i < 32 ? sa[i] : sbv[i - 32];
-                            p[e] = (i < nvalid) ? ex2_approx(fmaf(i2f(sij), c2, nb)) : 0.0f;
-                        }
-                        pw[w] = pack_e4m3x2(p[0], p[1]) | (pack_e4m3x2(p[2], p[3]) << 16);
-                    }
-                } else {
-#pragma unroll
-                    for (int w = 0; w < 16; ++w) pw[w] = 0u;
-                }
                 // the P buffer is free once the PV MMA of step gg-2 has completed
                 if (gg >= 2 && ok) ok = mbar_wait(bar(kBarPvDone + sb), ((gg >> 1) - 1) & 1, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
-                {
-                    uint8_t *prow = smem + kOffP + sb * kPTileBytes + row * 128;
+
+                // pass 2: P = e4m3(448 * 2^(S*c*log2e - mnew*log2e)), 32 keys at a time,
+                // written into the 128B-swizzled P tile (16-byte chunk k of row r at
+                // chunk position k ^ (r & 7))
+                const float c2 = c * kLog2e;
+                const float nb = kLog2_448 - mnew * kLog2e;
+                uint8_t *prow = smem + kOffP + sb * kPTileBytes + row * 128;
 #pragma unroll
-                    for (int cidx = 0; cidx < 4; ++cidx) {
-                        const int chunk = 4 * wg + cidx;
-                        *reinterpret_cast<uint4 *>(prow + ((chunk ^ (row & 7)) << 4)) =
-                            make_uint4(pw[4 * cidx], pw[4 * cidx + 1], pw[4 * cidx + 2], pw[4 * cidx + 3]);
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pw[8];
+                    if (j >= 0) {
+                        uint32_t xs[32];
+                        tmem_ld32_wait(taddr + 32 * h, xs);
+                        if (nvalid == 64) {
+#pragma unroll
+                            for (int w = 0; w < 8; ++w) {
+                                float y0, y1, y2, y3;
+                                fma2(y0, y1, i2f(xs[4 * w]), i2f(xs[4 * w + 1]), c2, c2, nb, nb);
+                                fma2(y2, y3, i2f(xs[4 * w + 2]), i2f(xs[4 * w + 3]), c2, c2, nb, nb);
+                                const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
+                                const float e2 = SA_POLY_OF_4 >= 2 ? exp2_poly(y2) : ex2_approx(y2);
+                                const float e3 = SA_POLY_OF_4 >= 1 ? exp2_poly(y3) : ex2_approx(y3);
+                                pw[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+                            }
+                        } else {
+#pragma unroll
+                            for (int w = 0; w < 8; ++w) {
+                                float e[4];
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    const int i = 32 * h + 4 * w + q;
+                                    e[q] = (i < nvalid) ? ex2_approx(fmaf(i2f(xs[4 * w + q]), c2, nb)) : 0.0f;
+                                }
+                                pw[w] = pack_e4m3x2(e[0], e[1]) | (pack_e4m3x2(e[2], e[3]) << 16);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) pw[w] = 0u;
                     }
+                    const int k0 = 4 * wg + 2 * h;
+                    *reinterpret_cast<uint4 *>(prow + ((k0 ^ (row & 7)) << 4)) =
+                        make_uint4(pw[0], pw[1], pw[2], pw[3]);
+                    *reinterpret_cast<uint4 *>(prow + (((k0 + 1) ^ (row & 7)) << 4)) =
+                        make_uint4(pw[4], pw[5], pw[6], pw[7]);
                 }
+                // S has been read for the last time: its buffer may take QK of step gg+2
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
+
                 // rescale O (and its row-sum column) when the running max grew
                 if (s > 0) {
                     const bool need = mnew > m;
@@ -387,11 +417,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t oa = tmem + lane_addr + kColO;
                             uint32_t r[32];
 #pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const uint32_t col = 64 * wg + 32 * h;
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const uint32_t col = 64 * wg + 32 * hh;
                                 tmem_ld32_wait(oa + col, r);
 #pragma unroll
-                                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                                for (int i = 0; i < 32; i += 2) {
+                                    float f0, f1;
+                                    mul2(f0, f1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), alpha, alpha);
+                                    r[i] = __float_as_uint(f0);
+                                    r[i + 1] = __float_as_uint(f1);
+                                }
                                 tmem_st32(oa + col, r);
                             }
                             uint32_t r8[8];
@@ -543,7 +578,21 @@ __global__ void debug_wait_timeout_kernel(unsigned long long timeout_ns)
     }
 }
 
+// Debug: the softmax's polynomial exp2 applied elementwise, for checking it against the
+// CUDA math library.
+__global__ void debug_exp2_poly_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = exp2_poly(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t st)
+{
+    debug_exp2_poly_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
 {

@@ -46,6 +46,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
 cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k, int BH,
                                 int Npad, int32_t *s_out, cudaStream_t st);
 cudaError_t launch_debug_wait_timeout(int timeout_us, cudaStream_t st);
+cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t st);
 // Reads and clears the device status word of the current device (synchronous).
 cudaError_t read_and_clear_status(int *status);
 

@@ -110,6 +110,12 @@ sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, 
  * status word and returns.  Exercises the failure path without faulting the GPU. */
 sa_status sa_debug_wait_timeout(int timeout_us, void *stream);
 
+/* Debug: y[i] = 2^x[i] computed by the attention kernel's polynomial exponential (the
+ * share of softmax exponentials moved off the MUFU pipe): Cody-Waite reduction and a
+ * fitted cubic, max relative error 7.5e-5 for -16 <= x <= 9; inputs below -16 are
+ * clamped to -16.  x, y: device fp32 [n]. */
+sa_status sa_debug_exp2_poly(const float *x, float *y, int n, void *stream);
+
 /* Synchronises the current device, returns and clears its device status word
  * (SA_OK or SA_ERR_DEVICE_TIMEOUT), or SA_ERR_CUDA if synchronisation failed. */
 sa_status sa_get_device_status(void);
