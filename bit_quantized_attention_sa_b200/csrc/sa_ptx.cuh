@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cstdio>
 #include <cuda_runtime.h>
 
 namespace sa {
@@ -78,6 +79,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             if (*abort) return false;
             if (globaltimer_ns() - t0 > SA_WAIT_LIMIT_NS) {
                 *abort = 1;
+                printf("sa: bounded wait expired: block %d thread %d barrier 0x%x parity %u\n",
+                       int(blockIdx.x), int(threadIdx.x), bar, parity);
                 return false;
             }
         }
@@ -286,6 +289,28 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16_wait(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait()
 {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -349,6 +374,32 @@ __device__ __forceinline__ float exp2_poly(float x)
     const float f = x - (t - kRound);
     const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, c0);
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two exp2_poly evaluations with the floating-point steps packed in pairs (f32x2).
+__device__ __forceinline__ void exp2_poly2(float &r0, float &r1, float x0, float x1)
+{
+    constexpr float kRound = 12582912.0f;
+    constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261115f, c3 = 0.05517177f;
+    x0 = fmaxf(x0, -16.0f);
+    x1 = fmaxf(x1, -16.0f);
+    float t0, t1, n0, n1, f0, f1, p0, p1;
+    fma2(t0, t1, x0, x1, 1.0f, 1.0f, kRound, kRound);     // t = x + 1.5*2^23
+    fma2(n0, n1, t0, t1, 1.0f, 1.0f, -kRound, -kRound);   // n = round(x)
+    fma2(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);           // f = x - n
+    fma2(p0, p1, f0, f1, c3, c3, c2, c2);
+    fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// max of three floats in one instruction (sm_100a)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ float ex2_approx(float x)

@@ -72,6 +72,7 @@ def test_quantized_entry_matches_full_forward(libsa, cuda_ok):
     q8, sq, k8, sk, _ = libsa.sa_quantize_qk(qd, kd)
     vt, sv = libsa.sa_quantize_v(vd)
     o2 = libsa.sa_attn_fwd_quantized(q8, sq, k8, sk, vt, sv, 777)
+    assert libsa.sa_get_device_status() == 0
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
 
 
