@@ -26,6 +26,7 @@ _I = ctypes.c_int
 _F = ctypes.c_float
 
 _lib.sa_quantize_qk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
+_lib.sa_quantize_qk_noalloc.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
 _lib.sa_quantize_v.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
@@ -40,7 +41,7 @@ _lib.sa_workspace_bytes.restype = ctypes.c_size_t
 _lib.sa_release_workspace.argtypes = []
 _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
-for _name in ("sa_quantize_qk", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_quantized",
+for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_quantized",
               "sa_debug_qk_s32", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
@@ -48,7 +49,7 @@ for _name in ("sa_quantize_qk", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_qua
 SA_OK = 0
 STATUS_NAMES = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED",
                 3: "SA_ERR_MISALIGNED", 4: "SA_ERR_CUDA", 5: "SA_ERR_OOM",
-                6: "SA_ERR_DEVICE_TIMEOUT"}
+                6: "SA_ERR_DEVICE_TIMEOUT", 7: "SA_ERR_SCRATCH_LIMIT"}
 
 
 class SAError(RuntimeError):

@@ -204,6 +204,23 @@ sa_status sa_quantize_qk(const void *q, const void *k, int B, int H, int N, int 
     return e == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
+sa_status sa_quantize_qk_noalloc(const void *q, const void *k, int B, int H, int N, int d,
+                                 int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                                 float *k_mean, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({q, k, q_i8, q_scale, k_i8, k_scale, k_mean})) != SA_OK) return r;
+    if (size_t(s.BH()) * size_t(s.nchunks()) * kD > kNoAllocPartialDoubles) return SA_ERR_SCRATCH_LIMIT;
+    if ((r = check_device()) != SA_OK) return r;
+    double *part = nullptr;
+    if (noalloc_kpart(&part) != cudaSuccess) return SA_ERR_CUDA;
+    cudaError_t e = launch_quantize_qk(q, k, s, q_i8, q_scale, k_i8, k_scale, k_mean, part,
+                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
 sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp8_t,
                         float *v_scale, void *stream)
 {
@@ -322,6 +339,7 @@ const char *sa_status_string(sa_status s)
     case SA_ERR_CUDA: return "SA_ERR_CUDA";
     case SA_ERR_OOM: return "SA_ERR_OOM";
     case SA_ERR_DEVICE_TIMEOUT: return "SA_ERR_DEVICE_TIMEOUT";
+    case SA_ERR_SCRATCH_LIMIT: return "SA_ERR_SCRATCH_LIMIT";
     }
     return "SA_ERR_UNKNOWN";
 }

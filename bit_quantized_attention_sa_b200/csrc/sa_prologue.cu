@@ -12,6 +12,8 @@
 // division followed by round-to-nearest-even (cvt.rni) or the e4m3 round-to-nearest-even
 // saturating conversion.  This file must not be built with fast-math or -prec-div=false.
 #include <cstdint>
+#include <mutex>
+
 #include <cuda_bf16.h>
 
 #include "sa_internal.h"
@@ -256,6 +258,34 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 }  // namespace
+
+// Scratch of sa_quantize_qk_noalloc: the fp64 per-chunk column sums of K, in a fixed
+// device array instead of the library's cudaMalloc'd workspace.  It lives for the whole
+// process on every device that loads the library, is shared by all calls (each call
+// overwrites every element it reads, so nothing needs clearing between calls), and two
+// such calls whose kernels overlap on one device race on it.
+static __device__ __align__(256) double g_noalloc_kpart[kNoAllocPartialDoubles];
+
+cudaError_t noalloc_kpart(double **out)
+{
+    // In host code the array's name is only a stand-in; the address the kernels must use
+    // is looked up once per device, with that device current.
+    static double *addr[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_kpart);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<double *>(ptr);
+    }
+    *out = addr[dev];
+    return cudaSuccess;
+}
 
 cudaError_t launch_quantize_qk(const void *q, const void *k, const Shape &s, int8_t *q_i8,
                                float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,

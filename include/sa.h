@@ -57,7 +57,8 @@ typedef enum {
     SA_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
     SA_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
     SA_ERR_OOM = 5,            /* the library workspace could not be allocated */
-    SA_ERR_DEVICE_TIMEOUT = 6  /* a device-side bounded wait expired */
+    SA_ERR_DEVICE_TIMEOUT = 6, /* a device-side bounded wait expired */
+    SA_ERR_SCRATCH_LIMIT = 7   /* the problem needs more than a fixed scratch array holds */
 } sa_status;
 
 /* Quantise Q and smooth + quantise K (the Q/K half of the prologue).
@@ -73,6 +74,24 @@ typedef enum {
 sa_status sa_quantize_qk(const void *q, const void *k, int B, int H, int N, int d,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, void *stream);
+
+/* sa_quantize_qk without any device allocation.  The method's pages have no counterpart
+ * for this; it exists for callers that cannot call cudaMalloc: code whose device memory is
+ * owned by a host framework or memory pool that has already reserved the device (so a
+ * library allocation would fail or fragment it), and latency-critical loops that cannot
+ * afford cudaMalloc's implicit synchronisation.  The library workspace that sa_quantize_qk
+ * grows on first use is replaced by a fixed 4 MiB device array compiled into the library
+ * (each GPU that loads the library holds it until the process exits).
+ * Arguments, outputs and results are exactly those of sa_quantize_qk.
+ * Limit: B * H * ceil(N / 1024) <= 4096 (e.g. 40 heads of up to 104,448 tokens); larger
+ * problems return SA_ERR_SCRATCH_LIMIT before any launch.
+ * The first call on each device looks up the array's device address (a synchronous
+ * runtime call), so make that first call before any stream capture.  All calls share the
+ * array: calls whose kernels overlap on the same device (e.g. on two streams) race on it
+ * and must be ordered by the caller.  No state carries over between calls. */
+sa_status sa_quantize_qk_noalloc(const void *q, const void *k, int B, int H, int N, int d,
+                                 int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                                 float *k_mean, void *stream);
 
 /* Quantise V to FP8 e4m3 per channel, stored transposed (the V half of the prologue).
  * Source: Video-Generation-101 research log 5.5 (FP8 P.V).
