@@ -10,8 +10,11 @@
 //   warp 8      producer: scans the tile's keep-mask row, pairs consecutive kept 64-key
 //               blocks into 128-key steps and TMA-loads the K (INT8) and V^T (FP8) tiles
 //               of each step into a STAGES-deep ring; loads the Q tile once per item.
-//   warp 9      MMA issuer (one thread): S = Q.K^T with tcgen05 kind::i8 into one of two
-//               tensor-memory S buffers; O += P.V with kind::f8f6f4 into the O buffer.
+//   warp 9      QK issuer (one thread): S = Q.K^T with tcgen05 kind::i8 into one of two
+//               tensor-memory S buffers.
+//   warp 10     PV issuer (one thread): O += P.V with kind::f8f6f4 into the O buffer.
+//               A tcgen05.mma holds its issuing warp for ~200 cycles whatever its shape,
+//               so the two streams are issued from two warps to overlap in the tensor core.
 //   warps 0-7   softmax: two warpgroups share each S tile by key half (warpgroup w owns
 //               the step's w-th 64-key block, so one K scale per thread); each thread owns
 //               one query row (its TMEM lane).  Row maxima are taken on int32 S and
@@ -38,10 +41,11 @@ __device__ int g_device_status;  // 0 = OK, 6 = a bounded wait expired
 
 namespace {
 
-constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kThreads = 352;
 constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
+constexpr int kWarpMmaQK = 9;
+constexpr int kWarpMmaPV = 10;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr int kOCols = 144;
@@ -78,7 +82,7 @@ constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, kOCols);
 // Of every 4 softmax exponentials, this many run as a polynomial on the FMA/ALU pipes
 // (exp2_poly) instead of the MUFU pipe, to balance the two.
 #ifndef SA_POLY_OF_4
-#define SA_POLY_OF_4 1
+#define SA_POLY_OF_4 0
 #endif
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         p[w] = (w < 16) ? 0x38383838u : 0u;
     }
     fence_proxy_async_smem();
-    if (warp == kWarpMma) tmem_alloc(sbase + kOffMisc, kTmemCols);
+    if (warp == kWarpMmaQK) tmem_alloc(sbase + kOffMisc, kTmemCols);
     if (warp == kWarpProducer && lane == 0) {
         prefetch_tmap(&tm_q);
         prefetch_tmap(&tm_k);
@@ -225,10 +229,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
         }
         if (lane == 0 && !ok) { *abort_flag = 1; record_timeout(); }
-    } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kWarpMmaQK) {
+        // ------------------------------------------------------------ QK issuer
+        // A tcgen05.mma blocks its issuing warp for roughly 200 cycles whatever its size,
+        // so S = Q.K^T and O += P.V are issued from two warps and overlap in the tensor
+        // core; each warp commits only its own operations.
         bool ok = true;
-        uint32_t g = 0, tl = 0, otile = 0;
+        uint32_t g = 0, tl = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tl) {
             const int bh = tile / nq, qt = tile % nq;
             const uint8_t *mrow = mask ? mask + (int64_t(bh) * nq + qt) * nk : nullptr;
@@ -238,11 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ok) ok = mbar_wait(bar(kBarQFull + qb), (tl >> 1) & 1, abort_flag);
                 tc_fence_after();
                 const uint32_t qa = sbase + kOffQ + qb * kQTileBytes;
-                auto issue_qk = [&](uint32_t gg) {
-                    const uint32_t st = gg % kStages, sb = gg & 1;
+                for (int s = 0; s < n; ++s) {
+                    const uint32_t gg = g + s, st = gg % kStages, sb = gg & 1;
                     if (ok) ok = mbar_wait(bar(kBarKvFull + st), (gg / kStages) & 1, abort_flag);
                     if (gg >= 2 && ok) ok = mbar_wait(bar(kBarSEmpty + sb), ((gg >> 1) - 1) & 1, abort_flag);
-                    if (!ok) return;
+                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t kb = sbase + kOffK + st * kKTileBytes;
                     const uint32_t dcol = tmem + (sb ? kColS1 : kColS0);
@@ -251,32 +258,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_i8(dcol, sdesc(qa + 32 * kk, 1024, SWZ_128B),
                                sdesc(kb + 32 * kk, 1024, SWZ_128B), kIdescQK, kk > 0);
                     tc_commit(bar(kBarSFull + sb));
-                };
-                if (n > 0) {
-                    issue_qk(g);
-                    if (n > 1) issue_qk(g + 1);
-                    for (int s = 0; s < n; ++s) {
-                        const uint32_t gg = g + s, st = gg % kStages, sb = gg & 1;
-                        if (ok) ok = mbar_wait(bar(kBarPFull + sb), (gg >> 1) & 1, abort_flag);
-                        if (s == 0 && otile >= 1 && ok)
-                            ok = mbar_wait(bar(kBarOEmpty), (otile - 1) & 1, abort_flag);
-                        if (ok) {
-                            tc_fence_after();
-                            const int nk_step = info[st].y >= 0 ? 4 : 2;
-                            const uint32_t pa = sbase + kOffP + sb * kPTileBytes;
-                            const uint32_t vb = sbase + kOffV + st * 2 * kVHalfBytes;
-                            for (int kk = 0; kk < nk_step; ++kk)
-                                mma_f8(tmem + kColO, sdesc(pa + 32 * kk, 1024, SWZ_128B),
-                                       sdesc(vb + (kk >> 1) * kVHalfBytes + 32 * (kk & 1), 512, SWZ_64B),
-                                       kIdescPV, (s > 0 || kk > 0) ? 1u : 0u);
-                            tc_commit(bar(kBarKvEmpty + st));
-                            tc_commit(bar(kBarPvDone + sb));
-                        }
-                        if (s + 2 < n) issue_qk(gg + 2);
-                    }
-                    if (ok) tc_commit(bar(kBarOFull));
                 }
                 if (ok) tc_commit(bar(kBarQEmpty + qb));
+            }
+            __syncwarp();
+            g += n;
+        }
+        if (lane == 0 && !ok) { *abort_flag = 1; record_timeout(); }
+    } else if (warp == kWarpMmaPV) {
+        // ------------------------------------------------------------ PV issuer
+        bool ok = true;
+        uint32_t g = 0, otile = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            const int bh = tile / nq, qt = tile % nq;
+            const uint8_t *mrow = mask ? mask + (int64_t(bh) * nq + qt) * nk : nullptr;
+            const int n = (count_kept(mrow, nk, lane) + 1) / 2;
+            if (lane == 0 && n > 0) {
+                for (int s = 0; s < n; ++s) {
+                    const uint32_t gg = g + s, st = gg % kStages, sb = gg & 1;
+                    // V of the stage (already complete: the softmax's P implies it) and P
+                    if (ok) ok = mbar_wait(bar(kBarKvFull + st), (gg / kStages) & 1, abort_flag);
+                    if (ok) ok = mbar_wait(bar(kBarPFull + sb), (gg >> 1) & 1, abort_flag);
+                    if (s == 0 && otile >= 1 && ok)
+                        ok = mbar_wait(bar(kBarOEmpty), (otile - 1) & 1, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const int nk_step = info[st].y >= 0 ? 4 : 2;
+                    const uint32_t pa = sbase + kOffP + sb * kPTileBytes;
+                    const uint32_t vb = sbase + kOffV + st * 2 * kVHalfBytes;
+                    for (int kk = 0; kk < nk_step; ++kk)
+                        mma_f8(tmem + kColO, sdesc(pa + 32 * kk, 1024, SWZ_128B),
+                               sdesc(vb + (kk >> 1) * kVHalfBytes + 32 * (kk & 1), 512, SWZ_64B),
+                               kIdescPV, (s > 0 || kk > 0) ? 1u : 0u);
+                    // QK of this step completed before its P existed, so the stage is free
+                    // once this PV completes
+                    tc_commit(bar(kBarKvEmpty + st));
+                    tc_commit(bar(kBarPvDone + sb));
+                }
+                if (ok) tc_commit(bar(kBarOFull));
             }
             __syncwarp();
             g += n;
@@ -316,94 +335,87 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int nvalid = j >= 0 ? min(64, N - 64 * j) : 0;
                 const uint32_t taddr = tmem + lane_addr + (sb ? kColS1 : kColS0) + 64 * wg;
 
-                // pass 1: row max of this half, on int32 S (the scale is positive)
+                // S of this half is read from tensor memory once and kept in registers;
+                // keys past the end of the sequence (last block only) are set to INT_MIN,
+                // so they drop out of the max and their weight underflows (their P bytes
+                // are also cleared below, which covers a zero scale)
                 float c = 0.0f, pmax = -INFINITY;
+                uint32_t a[32], b[32];
                 if (j >= 0) {
                     c = (sq * k_scale[int64_t(bh) * nk + j]) * sm_scale;
                     tc_fence_after();
-                    uint32_t a[32], b[32];
                     tmem_ld64_wait(taddr, a, b);
-                    int imax;
-                    if (nvalid == 64) {
-                        int acc[8];
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) acc[k] = max(int(a[k]), int(b[k]));
-#pragma unroll
-                        for (int i = 8; i < 32; i += 8)
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) acc[k] = max(acc[k], max(int(a[i + k]), int(b[i + k])));
-                        imax = max(max(max(acc[0], acc[1]), max(acc[2], acc[3])),
-                                   max(max(acc[4], acc[5]), max(acc[6], acc[7])));
-                    } else {
-                        imax = INT_MIN;
+                    if (nvalid < 64) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            if (i < nvalid) imax = max(imax, int(a[i]));
-                            if (i + 32 < nvalid) imax = max(imax, int(b[i]));
+                            if (i >= nvalid) a[i] = uint32_t(INT_MIN);
+                            if (i + 32 >= nvalid) b[i] = uint32_t(INT_MIN);
                         }
                     }
+                    // row max on int32 S (the scale is positive, so max commutes with it)
+                    int acc[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) acc[k] = max(int(a[k]), int(b[k]));
+#pragma unroll
+                    for (int i = 8; i < 32; i += 8)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) acc[k] = max(acc[k], max(int(a[i + k]), int(b[i + k])));
+                    const int imax = max(max(max(acc[0], acc[1]), max(acc[2], acc[3])),
+                                         max(max(acc[4], acc[5]), max(acc[6], acc[7])));
                     pmax = i2f(uint32_t(imax)) * c;
                 }
+                // S has been read: its buffer may take QK of step gg+2
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
+
                 float *x = xch + sb * 256;
                 x[wg * 128 + row] = pmax;
                 named_bar_sync(1 + wq, 64);
                 const float other = x[(wg ^ 1) * 128 + row];
                 const float mnew = fmaxf(m, fmaxf(pmax, other));
 
+                // P = e4m3(448 * 2^(S*c*log2e - mnew*log2e)) for this half: 64 keys -> 16 words
+                uint32_t pw[16];
+                if (j >= 0) {
+                    const float c2 = c * kLog2e;
+                    const float nb = kLog2_448 - mnew * kLog2e;
+#pragma unroll
+                    for (int w = 0; w < 16; ++w) {
+                        const uint32_t *src = w < 8 ? a : b;
+                        const int i = 4 * (w & 7);
+                        float y0, y1, y2, y3;
+                        fma2(y0, y1, i2f(src[i]), i2f(src[i + 1]), c2, c2, nb, nb);
+                        fma2(y2, y3, i2f(src[i + 2]), i2f(src[i + 3]), c2, c2, nb, nb);
+                        const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
+                        const float e2 = SA_POLY_OF_4 >= 2 ? exp2_poly(y2) : ex2_approx(y2);
+                        const float e3 = SA_POLY_OF_4 >= 1 ? exp2_poly(y3) : ex2_approx(y3);
+                        pw[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+                    }
+                    if (nvalid < 64) {
+#pragma unroll
+                        for (int w = 0; w < 16; ++w) {
+                            const int keep = nvalid - 4 * w;  // bytes of this word to keep
+                            pw[w] = keep >= 4 ? pw[w] : (keep <= 0 ? 0u : (pw[w] & ((1u << (8 * keep)) - 1u)));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int w = 0; w < 16; ++w) pw[w] = 0u;
+                }
                 // the P buffer is free once the PV MMA of step gg-2 has completed
                 if (gg >= 2 && ok) ok = mbar_wait(bar(kBarPvDone + sb), ((gg >> 1) - 1) & 1, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
-
-                // pass 2: P = e4m3(448 * 2^(S*c*log2e - mnew*log2e)), 32 keys at a time,
-                // written into the 128B-swizzled P tile (16-byte chunk k of row r at
-                // chunk position k ^ (r & 7))
-                const float c2 = c * kLog2e;
-                const float nb = kLog2_448 - mnew * kLog2e;
-                uint8_t *prow = smem + kOffP + sb * kPTileBytes + row * 128;
+                {
+                    // 128B-swizzled P tile: 16-byte chunk k of row r at position k ^ (r & 7)
+                    uint8_t *prow = smem + kOffP + sb * kPTileBytes + row * 128;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pw[8];
-                    if (j >= 0) {
-                        uint32_t xs[32];
-                        tmem_ld32_wait(taddr + 32 * h, xs);
-                        if (nvalid == 64) {
-#pragma unroll
-                            for (int w = 0; w < 8; ++w) {
-                                float y0, y1, y2, y3;
-                                fma2(y0, y1, i2f(xs[4 * w]), i2f(xs[4 * w + 1]), c2, c2, nb, nb);
-                                fma2(y2, y3, i2f(xs[4 * w + 2]), i2f(xs[4 * w + 3]), c2, c2, nb, nb);
-                                const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
-                                const float e2 = SA_POLY_OF_4 >= 2 ? exp2_poly(y2) : ex2_approx(y2);
-                                const float e3 = SA_POLY_OF_4 >= 1 ? exp2_poly(y3) : ex2_approx(y3);
-                                pw[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
-                            }
-                        } else {
-#pragma unroll
-                            for (int w = 0; w < 8; ++w) {
-                                float e[4];
-#pragma unroll
-                                for (int q = 0; q < 4; ++q) {
-                                    const int i = 32 * h + 4 * w + q;
-                                    e[q] = (i < nvalid) ? ex2_approx(fmaf(i2f(xs[4 * w + q]), c2, nb)) : 0.0f;
-                                }
-                                pw[w] = pack_e4m3x2(e[0], e[1]) | (pack_e4m3x2(e[2], e[3]) << 16);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int w = 0; w < 8; ++w) pw[w] = 0u;
+                    for (int cidx = 0; cidx < 4; ++cidx) {
+                        const int chunk = 4 * wg + cidx;
+                        *reinterpret_cast<uint4 *>(prow + ((chunk ^ (row & 7)) << 4)) =
+                            make_uint4(pw[4 * cidx], pw[4 * cidx + 1], pw[4 * cidx + 2], pw[4 * cidx + 3]);
                     }
-                    const int k0 = 4 * wg + 2 * h;
-                    *reinterpret_cast<uint4 *>(prow + ((k0 ^ (row & 7)) << 4)) =
-                        make_uint4(pw[0], pw[1], pw[2], pw[3]);
-                    *reinterpret_cast<uint4 *>(prow + (((k0 + 1) ^ (row & 7)) << 4)) =
-                        make_uint4(pw[4], pw[5], pw[6], pw[7]);
                 }
-                // S has been read for the last time: its buffer may take QK of step gg+2
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarSEmpty + sb));
-
                 // rescale O (and its row-sum column) when the running max grew
                 if (s > 0) {
                     const bool need = mnew > m;
@@ -415,20 +427,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                             const float alpha = need ? ex2_approx((m - mnew) * kLog2e) : 1.0f;
                             const uint32_t oa = tmem + lane_addr + kColO;
-                            uint32_t r[32];
+                            uint32_t r0[32], r1[32];
+                            tmem_ld64_wait(oa + 64 * wg, r0, r1);
 #pragma unroll
-                            for (int hh = 0; hh < 2; ++hh) {
-                                const uint32_t col = 64 * wg + 32 * hh;
-                                tmem_ld32_wait(oa + col, r);
-#pragma unroll
-                                for (int i = 0; i < 32; i += 2) {
-                                    float f0, f1;
-                                    mul2(f0, f1, __uint_as_float(r[i]), __uint_as_float(r[i + 1]), alpha, alpha);
-                                    r[i] = __float_as_uint(f0);
-                                    r[i + 1] = __float_as_uint(f1);
-                                }
-                                tmem_st32(oa + col, r);
+                            for (int i = 0; i < 32; i += 2) {
+                                float f0, f1;
+                                mul2(f0, f1, __uint_as_float(r0[i]), __uint_as_float(r0[i + 1]), alpha, alpha);
+                                r0[i] = __float_as_uint(f0);
+                                r0[i + 1] = __float_as_uint(f1);
+                                mul2(f0, f1, __uint_as_float(r1[i]), __uint_as_float(r1[i + 1]), alpha, alpha);
+                                r1[i] = __float_as_uint(f0);
+                                r1[i + 1] = __float_as_uint(f1);
                             }
+                            tmem_st32(oa + 64 * wg, r0);
+                            tmem_st32(oa + 64 * wg + 32, r1);
                             uint32_t r8[8];
                             tmem_ld8_wait(oa + 128 + 8 * wg, r8);
 #pragma unroll
@@ -444,39 +456,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarPFull + sb));
             }
-            // ---- epilogue: O = acc * scale_v / l, bf16
+            // ---- epilogue: O = acc * scale_v / l, bf16, 32 channels at a time
             if (ok) ok = mbar_wait(bar(kBarOFull), otile & 1, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
-            uint32_t oa[32], ob[32], lbits = 0;
             if (ok) {
                 tc_fence_after();
                 const uint32_t base = tmem + lane_addr + kColO;
-                tmem_ld32_wait(base + 64 * wg, oa);
-                tmem_ld32_wait(base + 64 * wg + 32, ob);
+                uint32_t lbits;
                 tmem_ld1_wait(base + 128, lbits);
+                const float l = __uint_as_float(lbits);
+                const float inv_l = l > 0.0f ? __frcp_rn(l) : 0.0f;  // a row with no kept key gives 0
+                const float *svp = v_scale + int64_t(bh) * kD + 64 * wg;
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t o[32];
+                    tmem_ld32_wait(base + 64 * wg + 32 * h, o);
+                    if (qrow < N) {
+#pragma unroll
+                        for (int cidx = 0; cidx < 4; ++cidx) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 8 * cidx + 2 * e;
+                                const float y0 = (__uint_as_float(o[i]) * svp[32 * h + i]) * inv_l;
+                                const float y1 = (__uint_as_float(o[i + 1]) * svp[32 * h + i + 1]) * inv_l;
+                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+                                w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                            reinterpret_cast<uint4 *>(orow)[4 * h + cidx] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarOEmpty));
-            if (ok && qrow < N) {
-                const float l = __uint_as_float(lbits);
-                const float *svp = v_scale + int64_t(bh) * kD + 64 * wg;
-#pragma unroll
-                for (int cidx = 0; cidx < 8; ++cidx) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 8 * cidx + 2 * e;
-                        const float a0 = __uint_as_float(i < 32 ? oa[i] : ob[i - 32]);
-                        const float a1 = __uint_as_float(i + 1 < 32 ? oa[i + 1] : ob[i + 1 - 32]);
-                        const float y0 = l > 0.0f ? __fdiv_rn(a0 * svp[i], l) : 0.0f;
-                        const float y1 = l > 0.0f ? __fdiv_rn(a1 * svp[i + 1], l) : 0.0f;
-                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
-                        w[e] = *reinterpret_cast<const uint32_t *>(&h2);
-                    }
-                    reinterpret_cast<uint4 *>(orow)[cidx] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
             g += n;
             ++otile;
         }
@@ -487,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == kWarpMma) tmem_dealloc(tmem, kTmemCols);
+    if (warp == kWarpMmaQK) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------------

@@ -4,7 +4,6 @@
 #pragma once
 
 #include <cstdint>
-#include <cstdio>
 #include <cuda_runtime.h>
 
 namespace sa {
@@ -79,8 +78,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             if (*abort) return false;
             if (globaltimer_ns() - t0 > SA_WAIT_LIMIT_NS) {
                 *abort = 1;
-                printf("sa: bounded wait expired: block %d thread %d barrier 0x%x parity %u\n",
-                       int(blockIdx.x), int(threadIdx.x), bar, parity);
                 return false;
             }
         }
