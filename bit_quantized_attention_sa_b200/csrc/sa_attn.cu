@@ -1,5 +1,9 @@
 // sa_attn.cu -- fused low-bit attention forward for sm_100a.
 //
+// Two kernels: attn_pairs_kernel (sa_attn_pairs.cuh) runs every call without a keep mask,
+// two query tiles per CTA; attn_fwd_kernel below runs masked calls, one query tile per
+// CTA, since two tiles generally keep different key blocks.
+//
 // Sources: "AIGC weekend special 5.10" section 1.2 Method, items (1) and (2)
 // (SageAttention2++ INT8 Q.K^T on tensor cores; SLA sparse attention on top);
 // "Video-Generation-101 research log" section 5.5 (INT Q.K^T, FP8 P.V); NetEase
@@ -600,6 +604,8 @@ __global__ void debug_exp2_poly_kernel(const float *__restrict__ x, float *__res
     if (i < n) y[i] = exp2_poly(x[i]);
 }
 
+#include "sa_attn_pairs.cuh"
+
 }  // namespace
 
 cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t st)
@@ -608,8 +614,35 @@ cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t
     return cudaGetLastError();
 }
 
+// Without a mask: two query tiles per CTA (attn_pairs_kernel).
+static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)
+{
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(attn_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(pairs::kSmemAlloc));
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int npairs = a.BH * ((a.nq + 1) / 2);
+    const int grid = npairs < sms ? npairs : sms;
+    attn_pairs_kernel<<<grid, pairs::kThreads, pairs::kSmemAlloc, st>>>(
+        a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale, a.v_scale, a.o, a.BH, a.N, a.Npad, a.nq, a.nk,
+        a.sm_scale);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
 {
+#ifndef SA_NO_PAIRS
+    if (!a.mask) return launch_attention_pairs(a, st);
+#endif
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -1,0 +1,506 @@
+// sa_attn_pairs.cuh -- the dense attention kernel: two query tiles per CTA.
+// Included by sa_attn.cu inside its anonymous namespace (shares its constants, the device
+// status word and the helpers above the include).
+//
+// Same computation as attn_fwd_kernel without a keep mask (every 64-key block kept, steps
+// of two consecutive blocks; "AIGC weekend special 5.10" section 1.2 Method item (1),
+// FlashAttention's tiled online softmax), organised for latency hiding:
+//   * A CTA takes a pair of 128-query tiles (A, B) of one head.  Both read the same K/V
+//     stream, so each K/V stage serves two tiles.
+//   * Warpgroup 0 (warps 0-3) runs the softmax, O rescaling and epilogue of tile A,
+//     warpgroup 1 (warps 4-7) those of tile B.  A thread owns one query row and all 128
+//     keys of a step, so the two warps on a scheduler work on independent rows: the
+//     exponentials of one overlap the tensor-memory loads, maxima and waits of the other,
+//     and no row maximum is exchanged between warps.
+//   * One S buffer in tensor memory serves both tiles in turn (QK_A(j), QK_B(j),
+//     QK_A(j+1), ...), which also staggers the two warpgroups by half a step; each tile
+//     has its own O accumulator (N = 144: 128 channels + the row-sum column fed by the
+//     constant e4m3 1.0 row of every V^T stage) and its own P tile in shared memory.
+//   * warp 8 producer (Q pair, K/V ring), warp 9 QK issuer, warp 10 PV issuer, warp 11
+//     idle (completes the third warpgroup).  Registers: 168 per thread at launch, the
+//     softmax warpgroups raise theirs to 232 (a whole 128-key row of S in registers) and
+//     the third lowers its to 40 (setmaxnreg): 2*232 + 40 <= 3*168.
+// Tensor memory: S [0,128), O_A [128,272), O_B [272,416).
+// Every mbarrier wait is bounded, as in attn_fwd_kernel.
+
+namespace pairs {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 384;
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMmaQK = 9;
+constexpr int kWarpMmaPV = 10;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;
+__host__ __device__ constexpr uint32_t col_o(int t) { return 128u + 144u * uint32_t(t); }
+
+constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;  // what __launch_bounds__(kThreads, 1) allows
+constexpr int kRegsSoftmax = 232, kRegsCtrl = 40;
+static_assert(128 * (2 * kRegsSoftmax + kRegsCtrl) <= kLaunchRegs * kThreads,
+              "the register split must fit the registers the block is launched with");
+
+constexpr uint32_t kOffQ = 0;                                    // Q_A, Q_B
+constexpr uint32_t kOffK = kOffQ + 2 * kQTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kKTileBytes;
+constexpr uint32_t kOffP = kOffV + kStages * 2 * kVHalfBytes;    // P_A, P_B
+constexpr uint32_t kOffBar = kOffP + 2 * kPTileBytes;
+constexpr int kBarQFull = 0, kBarQEmpty = 1, kBarKvFull = 2, kBarKvEmpty = kBarKvFull + kStages,
+              kBarSFull = kBarKvEmpty + kStages,  // [2]: per tile
+              kBarSEmpty = kBarSFull + 2, kBarPFull = kBarSEmpty + 1, kBarPvDone = kBarPFull + 2,
+              kBarOFull = kBarPvDone + 2, kBarOEmpty = kBarOFull + 2, kNumBars = kBarOEmpty + 2;
+constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;            // tmem base, abort flag
+constexpr uint32_t kSmemBytes = kOffMisc + 16;
+constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;               // 1024-B alignment slack
+
+static_assert(kOffK % 1024 == 0 && kOffV % 1024 == 0 && kOffP % 1024 == 0, "tile alignment");
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA");
+
+template <uint32_t NR>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(NR));
+}
+
+template <uint32_t NR>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(NR));
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane, without waiting: the
+// registers are valid only after tmem_wait_ld on the same array.
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// Orders later uses of r after a tcgen05.wait::ld (the array passes through the statement).
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// Four 32-column loads in flight, one wait: 128 columns [taddr, taddr + 128).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r0)[32], uint32_t (&r1)[32],
+                                           uint32_t (&r2)[32], uint32_t (&r3)[32])
+{
+    tmem_ld32_nowait(taddr, r0);
+    tmem_ld32_nowait(taddr + 32, r1);
+    tmem_ld32_nowait(taddr + 64, r2);
+    tmem_ld32_nowait(taddr + 96, r3);
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+    tmem_regs_ready(r0);
+    tmem_regs_ready(r1);
+    tmem_regs_ready(r2);
+    tmem_regs_ready(r3);
+}
+
+// Max of the 64 int32 values in two arrays of 32.
+__device__ __forceinline__ int max64x2(const uint32_t (&a)[32], const uint32_t (&b)[32])
+{
+    int acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = max(int(a[k]), int(b[k]));
+#pragma unroll
+    for (int i = 8; i < 32; i += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = max(acc[k], max(int(a[i + k]), int(b[i + k])));
+    return max(max(max(acc[0], acc[1]), max(acc[2], acc[3])), max(max(acc[4], acc[5]), max(acc[6], acc[7])));
+}
+
+// 32 keys of S (one array) -> 8 words of e4m3 P = 448 * 2^(S*c2 + nbias); bytes of keys at
+// or past `keep` (index within the array) are zero.
+__device__ __forceinline__ void p_words(const uint32_t (&v)[32], float c2, float nbias, int keep,
+                                        uint32_t (&pw)[8])
+{
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        float y0, y1, y2, y3;
+        fma2(y0, y1, i2f(v[4 * w]), i2f(v[4 * w + 1]), c2, c2, nbias, nbias);
+        fma2(y2, y3, i2f(v[4 * w + 2]), i2f(v[4 * w + 3]), c2, c2, nbias, nbias);
+        const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
+        const float e2 = SA_POLY_OF_4 >= 2 ? exp2_poly(y2) : ex2_approx(y2);
+        const float e3 = SA_POLY_OF_4 >= 1 ? exp2_poly(y3) : ex2_approx(y3);
+        pw[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+    }
+    if (keep < 32) {
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const int kb = keep - 4 * w;  // bytes of this word to keep
+            pw[w] = kb >= 4 ? pw[w] : (kb <= 0 ? 0u : (pw[w] & ((1u << (8 * kb)) - 1u)));
+        }
+    }
+}
+
+}  // namespace pairs
+
+__global__ void __launch_bounds__(pairs::kThreads, 1)
+    attn_pairs_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ q_scale,
+                      const float *__restrict__ k_scale, const float *__restrict__ v_scale,
+                      __nv_bfloat16 *__restrict__ out, int BH, int N, int Npad, int nq, int nk,
+                      float sm_scale)
+{
+    using pairs::kStages;
+    using pairs::kThreads;
+    using pairs::kWarpProducer;
+    using pairs::kWarpMmaQK;
+    using pairs::kWarpMmaPV;
+    using pairs::kTmemCols;
+    using pairs::kColS;
+    using pairs::col_o;
+    using pairs::kRegsSoftmax;
+    using pairs::kRegsCtrl;
+    using pairs::kOffQ;
+    using pairs::kOffK;
+    using pairs::kOffV;
+    using pairs::kOffP;
+    using pairs::kOffBar;
+    using pairs::kBarQFull;
+    using pairs::kBarQEmpty;
+    using pairs::kBarKvFull;
+    using pairs::kBarKvEmpty;
+    using pairs::kBarSFull;
+    using pairs::kBarSEmpty;
+    using pairs::kBarPFull;
+    using pairs::kBarPvDone;
+    using pairs::kBarOFull;
+    using pairs::kBarOEmpty;
+    using pairs::kOffMisc;
+    using pairs::setmaxnreg_inc;
+    using pairs::setmaxnreg_dec;
+    using pairs::tmem_ld128;
+    using pairs::max64x2;
+    using pairs::p_words;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile uint32_t *tmem_base_slot = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * uint32_t(i); };
+
+    // ---- set-up: barriers, constant V rows, tensor memory
+    if (threadIdx.x == 0) {
+        mbar_init(bar(kBarQFull), 1);
+        mbar_init(bar(kBarQEmpty), 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(kBarKvFull + s), 1);
+            mbar_init(bar(kBarKvEmpty + s), 1);
+        }
+        mbar_init(bar(kBarSEmpty), 4);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar(kBarSFull + t), 1);
+            mbar_init(bar(kBarPFull + t), 4);
+            mbar_init(bar(kBarPvDone + t), 1);
+            mbar_init(bar(kBarOFull + t), 1);
+            mbar_init(bar(kBarOEmpty + t), 4);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    // rows 128..143 of every V half tile: row 128 all e4m3 1.0 (0x38), the rest zero
+    for (int i = threadIdx.x; i < kStages * 2 * 16 * 16; i += kThreads) {
+        const int half = i / (16 * 16), w = i % (16 * 16);  // 16 rows x 16 words
+        uint32_t *p = reinterpret_cast<uint32_t *>(smem + kOffV + half * kVHalfBytes + kVHalfData);
+        p[w] = (w < 16) ? 0x38383838u : 0u;
+    }
+    fence_proxy_async_smem();
+    if (warp == kWarpMmaQK) tmem_alloc(sbase + kOffMisc, kTmemCols);
+    if (warp == kWarpProducer && lane == 0) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_base_slot;
+
+    const int npairs_h = (nq + 1) / 2, npairs = BH * npairs_h;
+    const int nsteps = (nk + 1) / 2;  // every block kept: blocks 2j and 2j+1 form step j
+    const bool odd_tail = (nk & 1) != 0;  // the last step then has one block
+
+    if (warp >= kWarpProducer) {
+        setmaxnreg_dec<kRegsCtrl>();
+        if (warp == kWarpProducer && lane == 0) {
+            // ------------------------------------------------------------ producer
+            bool ok = true;
+            uint32_t g = 0, pl = 0;
+            for (int p = blockIdx.x; p < npairs; p += gridDim.x, ++pl) {
+                const int bh = p / npairs_h, qa = 2 * (p % npairs_h);
+                const bool hasb = qa + 1 < nq;
+                if (pl >= 1 && ok) ok = mbar_wait(bar(kBarQEmpty), (pl - 1) & 1, abort_flag);
+                if (ok) {
+                    mbar_arrive_expect_tx(bar(kBarQFull), (hasb ? 2u : 1u) * kQTileBytes);
+                    tma_load_2d(sbase + kOffQ, &tm_q, bar(kBarQFull), 0, bh * Npad + qa * 128);
+                    if (hasb)
+                        tma_load_2d(sbase + kOffQ + kQTileBytes, &tm_q, bar(kBarQFull), 0, bh * Npad + qa * 128 + 128);
+                }
+                for (int j = 0; j < nsteps && ok; ++j, ++g) {
+                    const uint32_t st = g % kStages;
+                    const bool two = !(odd_tail && j == nsteps - 1);
+                    if (g >= kStages) ok = mbar_wait(bar(kBarKvEmpty + st), ((g / kStages) - 1) & 1, abort_flag);
+                    if (!ok) break;
+                    const uint32_t kb = sbase + kOffK + st * kKTileBytes;
+                    const uint32_t vb = sbase + kOffV + st * 2 * kVHalfBytes;
+                    mbar_arrive_expect_tx(bar(kBarKvFull + st), (two ? 2u : 1u) * (kKHalfBytes + kVHalfData));
+                    tma_load_2d(kb, &tm_k, bar(kBarKvFull + st), 0, bh * Npad + 128 * j);
+                    tma_load_2d(vb, &tm_v, bar(kBarKvFull + st), 128 * j, bh * 128);
+                    if (two) {
+                        tma_load_2d(kb + kKHalfBytes, &tm_k, bar(kBarKvFull + st), 0, bh * Npad + 128 * j + 64);
+                        tma_load_2d(vb + kVHalfBytes, &tm_v, bar(kBarKvFull + st), 128 * j + 64, bh * 128);
+                    }
+                }
+            }
+            if (!ok) { *abort_flag = 1; record_timeout(); }
+        } else if (warp == kWarpMmaQK && lane == 0) {
+            // ------------------------------------------------------------ QK issuer
+            // S_A(j), S_B(j), S_A(j+1), ... through the one S buffer
+            bool ok = true;
+            uint32_t g = 0, u = 0, pl = 0;
+            for (int p = blockIdx.x; p < npairs && ok; p += gridDim.x, ++pl) {
+                const int qa = 2 * (p % npairs_h);
+                const int ntile = qa + 1 < nq ? 2 : 1;
+                ok = mbar_wait(bar(kBarQFull), pl & 1, abort_flag);
+                tc_fence_after();
+                for (int j = 0; j < nsteps && ok; ++j, ++g) {
+                    const uint32_t st = g % kStages;
+                    ok = mbar_wait(bar(kBarKvFull + st), (g / kStages) & 1, abort_flag);
+                    const uint32_t kb = sbase + kOffK + st * kKTileBytes;
+                    for (int t = 0; t < ntile && ok; ++t, ++u) {
+                        if (u >= 1) ok = mbar_wait(bar(kBarSEmpty), (u - 1) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t qaddr = sbase + kOffQ + uint32_t(t) * kQTileBytes;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_i8(tmem + kColS, sdesc(qaddr + 32 * kk, 1024, SWZ_128B),
+                                   sdesc(kb + 32 * kk, 1024, SWZ_128B), kIdescQK, kk > 0);
+                        tc_commit(bar(kBarSFull + t));
+                    }
+                }
+                if (ok) tc_commit(bar(kBarQEmpty));
+            }
+            if (!ok) { *abort_flag = 1; record_timeout(); }
+        } else if (warp == kWarpMmaPV && lane == 0) {
+            // ------------------------------------------------------------ PV issuer
+            bool ok = true;
+            uint32_t g = 0, c[2] = {0, 0}, o[2] = {0, 0};
+            for (int p = blockIdx.x; p < npairs && ok; p += gridDim.x) {
+                const int qa = 2 * (p % npairs_h);
+                const int ntile = qa + 1 < nq ? 2 : 1;
+                for (int j = 0; j < nsteps && ok; ++j, ++g) {
+                    const uint32_t st = g % kStages;
+                    const int nkk = (odd_tail && j == nsteps - 1) ? 2 : 4;  // K = 64 or 128 keys
+                    ok = mbar_wait(bar(kBarKvFull + st), (g / kStages) & 1, abort_flag);
+                    const uint32_t vb = sbase + kOffV + st * 2 * kVHalfBytes;
+                    for (int t = 0; t < ntile && ok; ++t) {
+                        ok = mbar_wait(bar(kBarPFull + t), c[t] & 1, abort_flag);
+                        if (ok && j == 0 && o[t] >= 1) ok = mbar_wait(bar(kBarOEmpty + t), (o[t] - 1) & 1, abort_flag);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t pa = sbase + kOffP + uint32_t(t) * kPTileBytes;
+                        for (int kk = 0; kk < nkk; ++kk)
+                            mma_f8(tmem + col_o(t), sdesc(pa + 32 * kk, 1024, SWZ_128B),
+                                   sdesc(vb + (kk >> 1) * kVHalfBytes + 32 * (kk & 1), 512, SWZ_64B),
+                                   kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                        tc_commit(bar(kBarPvDone + t));
+                        ++c[t];
+                    }
+                    // QK of this step completed before its P existed, so the stage is free
+                    // once the PVs of this step complete
+                    if (ok) tc_commit(bar(kBarKvEmpty + st));
+                }
+                for (int t = 0; t < ntile && ok; ++t) {
+                    tc_commit(bar(kBarOFull + t));
+                    ++o[t];
+                }
+            }
+            if (!ok) { *abort_flag = 1; record_timeout(); }
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax, tile t
+        setmaxnreg_inc<kRegsSoftmax>();
+        const int t = warp >> 2;                 // 0: tile A, 1: tile B
+        const int wq = warp & 3;                 // TMEM lane quarter
+        const int row = wq * 32 + lane;          // query row within the tile
+        const uint32_t lane_addr = uint32_t(wq * 32) << 16;
+        const uint32_t sa = tmem + lane_addr + kColS;
+        const uint32_t oa = tmem + lane_addr + col_o(t);
+        uint8_t *prow = smem + kOffP + uint32_t(t) * kPTileBytes + row * 128;
+        bool ok = true;
+        uint32_t c = 0, o = 0;  // steps and tiles this warpgroup has processed
+        for (int p = blockIdx.x; p < npairs; p += gridDim.x) {
+            const int bh = p / npairs_h, qt = 2 * (p % npairs_h) + t;
+            if (qt >= nq) continue;  // tile B of the last pair of an odd tile count
+            const int qrow = qt * 128 + row;
+            const float sq = q_scale[int64_t(bh) * nq + qt];
+            const float *ksrow = k_scale + int64_t(bh) * nk;
+            float m = -INFINITY;
+            for (int j = 0; j < nsteps; ++j, ++c) {
+                const bool two = !(odd_tail && j == nsteps - 1);
+                const float ks0 = ksrow[2 * j], ks1 = two ? ksrow[2 * j + 1] : 0.0f;
+                const int nv0 = min(64, N - 128 * j), nv1 = two ? min(64, N - 128 * j - 64) : 0;
+                if (ok) ok = mbar_wait(bar(kBarSFull + t), c & 1, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+
+                // S of this step, all 128 keys of the row, read once; then the buffer goes
+                // to the other tile's QK
+                uint32_t s0[32], s1[32], s2[32], s3[32];
+                if (ok) {
+                    tc_fence_after();
+                    tmem_ld128(sa, s0, s1, s2, s3);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarSEmpty));
+
+                // keys past the end of the sequence (last block only) drop out of the max
+                // (their P bytes are cleared below)
+                if (nv0 < 64) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (i >= nv0) s0[i] = uint32_t(INT_MIN);
+                        if (i + 32 >= nv0) s1[i] = uint32_t(INT_MIN);
+                    }
+                }
+                if (two && nv1 < 64) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (i >= nv1) s2[i] = uint32_t(INT_MIN);
+                        if (i + 32 >= nv1) s3[i] = uint32_t(INT_MIN);
+                    }
+                }
+                // row max on int32 S per block (each scale is positive, so max commutes)
+                const float c0 = (sq * ks0) * sm_scale, c1 = (sq * ks1) * sm_scale;
+                float pmax = i2f(uint32_t(max64x2(s0, s1))) * c0;
+                if (two) pmax = fmaxf(pmax, i2f(uint32_t(max64x2(s2, s3))) * c1);
+                const float mnew = fmaxf(m, pmax);
+
+                // P = e4m3(448 * 2^(S*c*log2e - mnew*log2e)), 8 words per 32 keys
+                const float nbias = kLog2_448 - mnew * kLog2e;
+                uint32_t pw[4][8];
+                p_words(s0, c0 * kLog2e, nbias, nv0, pw[0]);
+                p_words(s1, c0 * kLog2e, nbias, nv0 - 32, pw[1]);
+                if (two) {
+                    p_words(s2, c1 * kLog2e, nbias, nv1, pw[2]);
+                    p_words(s3, c1 * kLog2e, nbias, nv1 - 32, pw[3]);
+                } else {
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) pw[2][w] = pw[3][w] = 0u;
+                }
+
+                // the P tile and O are free once the PV of the previous step completed
+                if (c >= 1 && ok) ok = mbar_wait(bar(kBarPvDone + t), (c - 1) & 1, abort_flag);
+                ok = __all_sync(0xffffffffu, ok);
+                // 128B-swizzled P tile: 16-byte chunk k of row r at position k ^ (r & 7)
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    *reinterpret_cast<uint4 *>(prow + ((k ^ (row & 7)) << 4)) =
+                        make_uint4(pw[k >> 1][4 * (k & 1)], pw[k >> 1][4 * (k & 1) + 1],
+                                   pw[k >> 1][4 * (k & 1) + 2], pw[k >> 1][4 * (k & 1) + 3]);
+
+                // rescale O (and its row-sum column) when the running max grew
+                if (j > 0) {
+                    const bool need = mnew > m;
+                    if (__any_sync(0xffffffffu, need) && ok) {
+                        tc_fence_after();
+                        const float alpha = need ? ex2_approx((m - mnew) * kLog2e) : 1.0f;
+#pragma unroll 1
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t r0[32], r1[32];
+                            tmem_ld64_wait(oa + 64 * h, r0, r1);
+#pragma unroll
+                            for (int i = 0; i < 32; i += 2) {
+                                float f0, f1;
+                                mul2(f0, f1, __uint_as_float(r0[i]), __uint_as_float(r0[i + 1]), alpha, alpha);
+                                r0[i] = __float_as_uint(f0);
+                                r0[i + 1] = __float_as_uint(f1);
+                                mul2(f0, f1, __uint_as_float(r1[i]), __uint_as_float(r1[i + 1]), alpha, alpha);
+                                r1[i] = __float_as_uint(f0);
+                                r1[i + 1] = __float_as_uint(f1);
+                            }
+                            tmem_st32(oa + 64 * h, r0);
+                            tmem_st32(oa + 64 * h + 32, r1);
+                        }
+                        uint32_t r8[8];
+                        tmem_ld8_wait(oa + 128, r8);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) r8[i] = __float_as_uint(__uint_as_float(r8[i]) * alpha);
+                        tmem_st8(oa + 128, r8);
+                        tmem_st_wait();
+                    }
+                }
+                m = mnew;
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarPFull + t));
+            }
+            // ---- epilogue: O = acc * scale_v / l, bf16, 32 channels at a time
+            if (ok) ok = mbar_wait(bar(kBarOFull + t), o & 1, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+                tc_fence_after();
+                uint32_t lbits;
+                tmem_ld1_wait(oa + 128, lbits);
+                const float l = __uint_as_float(lbits);
+                const float inv_l = l > 0.0f ? __frcp_rn(l) : 0.0f;
+                const float *svp = v_scale + int64_t(bh) * kD;
+                __nv_bfloat16 *orow = out + (int64_t(bh) * N + qrow) * kD;
+#pragma unroll 1
+                for (int h = 0; h < 4; ++h) {
+                    uint32_t ov[32];
+                    tmem_ld32_wait(oa + 32 * h, ov);
+                    if (qrow < N) {
+#pragma unroll
+                        for (int cidx = 0; cidx < 4; ++cidx) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int i = 8 * cidx + 2 * e;
+                                const float y0 = (__uint_as_float(ov[i]) * svp[32 * h + i]) * inv_l;
+                                const float y1 = (__uint_as_float(ov[i + 1]) * svp[32 * h + i + 1]) * inv_l;
+                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
+                                w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                            reinterpret_cast<uint4 *>(orow)[4 * h + cidx] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarOEmpty + t));
+            ++o;
+        }
+        if (lane == 0 && !ok) { *abort_flag = 1; record_timeout(); }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMmaQK) tmem_dealloc(tmem, kTmemCols);
+}
