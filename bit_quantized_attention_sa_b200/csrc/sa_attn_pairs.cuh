@@ -365,16 +365,12 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                 if (ok) ok = mbar_wait(bar(kBarSFull + t), c & 1, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
 
-                // S of this step, all 128 keys of the row, read once; then the buffer goes
-                // to the other tile's QK
+                // S of this step, all 128 keys of the row, read once
                 uint32_t s0[32], s1[32], s2[32], s3[32];
                 if (ok) {
                     tc_fence_after();
                     tmem_ld128(sa, s0, s1, s2, s3);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarSEmpty));
 
                 // keys past the end of the sequence (last block only) drop out of the max
                 // (their P bytes are cleared below)
@@ -397,12 +393,21 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                 float pmax = i2f(uint32_t(max64x2(s0, s1))) * c0;
                 if (two) pmax = fmaxf(pmax, i2f(uint32_t(max64x2(s2, s3))) * c1);
                 const float mnew = fmaxf(m, pmax);
+                // the S buffer goes to the other tile's QK only now, after the maximum: this
+                // delays the other warpgroup by about that long, so that its exponentials
+                // tend to run while this one loads, stores and waits (measured at 720p:
+                // 97.2 ms, against 103.4 ms for a release right after the load and 114 ms
+                // for one after the first exponentials)
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarSEmpty));
 
                 // P = e4m3(448 * 2^(S*c*log2e - mnew*log2e)), 8 words per 32 keys
                 const float nbias = kLog2_448 - mnew * kLog2e;
                 uint32_t pw[4][8];
                 p_words(s0, c0 * kLog2e, nbias, nv0, pw[0]);
                 p_words(s1, c0 * kLog2e, nbias, nv0 - 32, pw[1]);
+
                 if (two) {
                     p_words(s2, c1 * kLog2e, nbias, nv1, pw[2]);
                     p_words(s3, c1 * kLog2e, nbias, nv1 - 32, pw[3]);
