@@ -51,17 +51,26 @@ def measured_peak():
         return 2.0 * 1590.0, "fallback 1.59 PFLOP/s bf16 x 2 (nominal 8-bit/bf16 ratio)"
 
 
-def recorded_traffic():
+KERNEL_SOURCES = ("sa_attn.cu", "sa_attn_pairs.cuh")
+
+
+def kernel_source_sha256():
+    """sha256 over the attention kernels' source files, in order."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "bit_quantized_attention_sa_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel sources and for this kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
-    src = os.path.join(ROOT, "bit_quantized_attention_sa_b200", "csrc", "sa_attn.cu")
     try:
         with open(p) as f:
             rec = json.load(f)
-        with open(src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()
-        if rec.get("sa_attn_cu_sha256") != h:
+        if rec.get("kernel_sources_sha256") != kernel_source_sha256() or rec.get("kernel") != kernel:
             return None
         return rec
     except Exception:
@@ -293,7 +302,8 @@ def main():
     value = ops_rank * world / t_step / 1e12
     peak, peak_src = measured_peak()
     achieved = ops_rank / t_attn / 1e12
-    traffic = recorded_traffic()
+    kernel = "attn_fwd_kernel" if w.mask_density is not None else "attn_pairs_kernel"
+    traffic = recorded_traffic(kernel)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -312,7 +322,7 @@ def main():
                        "step": "sa_attn_fwd: K mean + Q/K INT8 + V FP8 prologue + fused attention",
                        "l2": "inputs larger than L2 (each bf16 tensor %.0f MB)" % (h2d / 3 / 1e6),
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel",
+            "roofline": {"bound": "tensor", "kernel": kernel,
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_source": peak_src,
                          "frac_of_datasheet_4500": achieved / DATASHEET_TOPS,
