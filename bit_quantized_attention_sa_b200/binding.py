@@ -29,6 +29,7 @@ _lib.sa_quantize_qk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
 _lib.sa_quantize_qk_noalloc.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]
 _lib.sa_quantize_v.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
+_lib.sa_attn_fwd_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
 _lib.sa_debug_wait_timeout.argtypes = [_I, _P]
@@ -41,7 +42,8 @@ _lib.sa_workspace_bytes.restype = ctypes.c_size_t
 _lib.sa_release_workspace.argtypes = []
 _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
-for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_quantized",
+for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
+              "sa_attn_fwd_quantized",
               "sa_debug_qk_s32", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
@@ -156,6 +158,33 @@ def sa_attn_fwd(q, k, v, sm_scale: float | None = None, block_mask=None, out=Non
     _need(o, torch.bfloat16, "out")
     _check(_lib.sa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, float(sm_scale),
                             _ptr(m), _stream(q.device)), "sa_attn_fwd")
+    return o
+
+
+def sa_attn_fwd_host(q, k, v, out=None, sm_scale: float | None = None, block_mask=None,
+                     stream: torch.cuda.Stream | None = None):
+    """bf16 [B,H,N,d] CPU tensors (pin_memory() for overlapped copies) -> bf16 CPU O.  The
+    copies and the computation are enqueued on `stream` (default: the current CUDA stream);
+    O is complete once that stream reaches this point (e.g. after stream.synchronize()), and
+    the input tensors must be kept alive until then."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous CPU bf16 tensor")
+    B, H, N, d = _dims(q)
+    if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
+        raise ValueError("q, k, v shapes differ")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if block_mask is not None:
+        if block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous() \
+                or tuple(block_mask.shape) != (B, H, -(-N // 128), -(-N // 64)):
+            raise ValueError("block_mask must be a contiguous CPU uint8 [B, H, ceil(N/128), ceil(N/64)]")
+    o = torch.empty_like(q, pin_memory=q.is_pinned()) if out is None else out
+    if o.is_cuda or o.dtype != torch.bfloat16 or not o.is_contiguous() or o.shape != q.shape:
+        raise ValueError("out must be a contiguous CPU bf16 tensor shaped like q")
+    st = torch.cuda.current_stream() if stream is None else stream
+    _check(_lib.sa_attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, float(sm_scale),
+                                 _ptr(block_mask), ctypes.c_void_p(st.cuda_stream)), "sa_attn_fwd_host")
     return o
 
 

@@ -2,6 +2,7 @@
 // grow-only workspace, TMA tensor-map encoding and launch sequencing on the caller's
 // stream.  No entry point synchronises except sa_get_device_status and
 // sa_release_workspace.
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -180,6 +181,143 @@ static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t 
     return launch_attention(a, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
+// Prologue into the library workspace, then the fused attention kernel (validated args).
+static sa_status attn_fwd_device(const void *q, const void *k, const void *v, void *o,
+                                 const Shape &s, float sm_scale, const uint8_t *block_mask,
+                                 cudaStream_t st)
+{
+    const WsLayout L = ws_layout(s);
+    uint8_t *ws = nullptr;
+    sa_status r = get_workspace(L.total, &ws);
+    if (r != SA_OK) return r;
+    int8_t *q8 = reinterpret_cast<int8_t *>(ws + L.q8);
+    int8_t *k8 = reinterpret_cast<int8_t *>(ws + L.k8);
+    uint8_t *v8 = ws + L.v8;
+    float *sq = reinterpret_cast<float *>(ws + L.sq);
+    float *sk = reinterpret_cast<float *>(ws + L.sk);
+    float *sv = reinterpret_cast<float *>(ws + L.sv);
+    if (launch_quantize_qk(q, k, s, q8, sq, k8, sk, reinterpret_cast<float *>(ws + L.kmean),
+                           reinterpret_cast<double *>(ws + L.kpart), st) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st) !=
+        cudaSuccess)
+        return SA_ERR_CUDA;
+    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st);
+}
+
+// ------------------------------------------------------------------ host-buffer pipeline
+//
+// sa_attn_fwd_host: the heads (b, h) are independent, so the B*H heads are cut into chunks
+// of consecutive heads; the upload of chunk c+1 and the download of chunk c-1 run on two
+// library streams while chunk c is computed on the caller's stream.  Two staging slots per
+// device alternate between chunks; events order each slot's reuse:
+//   upload(c)   waits compute(c-2)   (its inputs were read)
+//   compute(c)  waits upload(c) and download(c-2) (its output slot was copied out)
+//   download(c) waits compute(c)
+// and the caller's stream finally waits for both slots' last download.
+
+constexpr size_t kHostChunkTensorBytes = size_t(64) << 20;  // target bytes of q per chunk
+
+struct HostPipe {
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t entry = nullptr, in[2] = {nullptr, nullptr}, comp[2] = {nullptr, nullptr},
+                out[2] = {nullptr, nullptr};
+    void *buf = nullptr;
+    size_t bytes = 0;
+};
+static HostPipe g_hp[64];
+static std::mutex g_hp_mutex;
+
+static sa_status host_pipe_init(HostPipe &P)
+{
+    if (P.h2d) return SA_OK;
+    if (cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&P.entry, cudaEventDisableTiming) != cudaSuccess)
+        return SA_ERR_CUDA;
+    for (int i = 0; i < 2; ++i)
+        if (cudaEventCreateWithFlags(&P.in[i], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&P.comp[i], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&P.out[i], cudaEventDisableTiming) != cudaSuccess)
+            return SA_ERR_CUDA;
+    return SA_OK;
+}
+
+static sa_status attn_fwd_host_pipeline(const void *q, const void *k, const void *v, void *o,
+                                        const Shape &s, float sm_scale, const uint8_t *mask,
+                                        cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_hp_mutex);
+    HostPipe &P = g_hp[dev];
+    sa_status r = host_pipe_init(P);
+    if (r != SA_OK) return r;
+
+    const int64_t BH = s.BH();
+    const size_t head_bytes = size_t(s.N) * kD * 2;                  // one head of q (bf16)
+    const size_t head_mask = size_t(s.nq()) * size_t(s.nk());        // one head of the mask
+    const int64_t hc = std::max<int64_t>(1, std::min<int64_t>(BH, int64_t(kHostChunkTensorBytes / head_bytes)));
+    const size_t t_bytes = align256(size_t(hc) * head_bytes);
+    const size_t m_bytes = mask ? align256(size_t(hc) * head_mask) : 0;
+    const size_t slot = 4 * t_bytes + m_bytes;
+    if (P.bytes < 2 * slot) {
+        if (P.buf) {
+            // earlier calls may still use the old staging buffer
+            if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;
+            cudaFree(P.buf);
+            P.buf = nullptr;
+            P.bytes = 0;
+        }
+        if (cudaMalloc(&P.buf, 2 * slot) != cudaSuccess) {
+            cudaGetLastError();
+            return SA_ERR_OOM;
+        }
+        P.bytes = 2 * slot;
+    }
+    const uint8_t *hq = static_cast<const uint8_t *>(q), *hk = static_cast<const uint8_t *>(k),
+                  *hv = static_cast<const uint8_t *>(v);
+    uint8_t *ho = static_cast<uint8_t *>(o);
+    // the inputs may be written by work already enqueued on the caller's stream
+    if (cudaEventRecord(P.entry, st) != cudaSuccess || cudaStreamWaitEvent(P.h2d, P.entry, 0) != cudaSuccess)
+        return SA_ERR_CUDA;
+    int last[2] = {0, 0};
+    for (int64_t h0 = 0, c = 0; h0 < BH; h0 += hc, ++c) {
+        const int i = int(c & 1);
+        const int64_t hn = std::min<int64_t>(hc, BH - h0);
+        const size_t nb = size_t(hn) * head_bytes, off = size_t(h0) * head_bytes;
+        uint8_t *base = static_cast<uint8_t *>(P.buf) + size_t(i) * slot;
+        uint8_t *dq = base, *dk = base + t_bytes, *dv = base + 2 * t_bytes, *dout = base + 3 * t_bytes;
+        uint8_t *dm = mask ? base + 4 * t_bytes : nullptr;
+        bool ok = cudaStreamWaitEvent(P.h2d, P.comp[i], 0) == cudaSuccess &&
+                  cudaMemcpyAsync(dq, hq + off, nb, cudaMemcpyHostToDevice, P.h2d) == cudaSuccess &&
+                  cudaMemcpyAsync(dk, hk + off, nb, cudaMemcpyHostToDevice, P.h2d) == cudaSuccess &&
+                  cudaMemcpyAsync(dv, hv + off, nb, cudaMemcpyHostToDevice, P.h2d) == cudaSuccess &&
+                  (!mask || cudaMemcpyAsync(dm, mask + size_t(h0) * head_mask, size_t(hn) * head_mask,
+                                            cudaMemcpyHostToDevice, P.h2d) == cudaSuccess) &&
+                  cudaEventRecord(P.in[i], P.h2d) == cudaSuccess &&
+                  cudaStreamWaitEvent(st, P.in[i], 0) == cudaSuccess &&
+                  cudaStreamWaitEvent(st, P.out[i], 0) == cudaSuccess;
+        if (!ok) return SA_ERR_CUDA;
+        Shape sc;
+        sc.B = 1;
+        sc.H = int(hn);
+        sc.N = s.N;
+        r = attn_fwd_device(dq, dk, dv, dout, sc, sm_scale, dm, st);
+        if (r != SA_OK) return r;
+        ok = cudaEventRecord(P.comp[i], st) == cudaSuccess &&
+             cudaStreamWaitEvent(P.d2h, P.comp[i], 0) == cudaSuccess &&
+             cudaMemcpyAsync(ho + off, dout, nb, cudaMemcpyDeviceToHost, P.d2h) == cudaSuccess &&
+             cudaEventRecord(P.out[i], P.d2h) == cudaSuccess;
+        if (!ok) return SA_ERR_CUDA;
+        last[i] = 1;
+    }
+    // the call is complete on the caller's stream once the outputs are in host memory
+    for (int i = 0; i < 2; ++i)
+        if (last[i] && cudaStreamWaitEvent(st, P.out[i], 0) != cudaSuccess) return SA_ERR_CUDA;
+    return SA_OK;
+}
+
 }  // namespace sa
 
 using namespace sa;
@@ -247,23 +385,19 @@ sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int 
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
-    const WsLayout L = ws_layout(s);
-    uint8_t *ws = nullptr;
-    if ((r = get_workspace(L.total, &ws)) != SA_OK) return r;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int8_t *q8 = reinterpret_cast<int8_t *>(ws + L.q8);
-    int8_t *k8 = reinterpret_cast<int8_t *>(ws + L.k8);
-    uint8_t *v8 = ws + L.v8;
-    float *sq = reinterpret_cast<float *>(ws + L.sq);
-    float *sk = reinterpret_cast<float *>(ws + L.sk);
-    float *sv = reinterpret_cast<float *>(ws + L.sv);
-    if (launch_quantize_qk(q, k, s, q8, sq, k8, sk, reinterpret_cast<float *>(ws + L.kmean),
-                           reinterpret_cast<double *>(ws + L.kpart), st) != cudaSuccess)
-        return SA_ERR_CUDA;
-    if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st) !=
-        cudaSuccess)
-        return SA_ERR_CUDA;
-    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st);
+    return attn_fwd_device(q, k, v, o, s, sm_scale, block_mask, static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_attn_fwd_host(const void *q, const void *k, const void *v, void *o, int B, int H,
+                           int N, int d, float sm_scale, const uint8_t *block_mask, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
+    if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    return attn_fwd_host_pipeline(q, k, v, o, s, sm_scale, block_mask, static_cast<cudaStream_t>(stream));
 }
 
 sa_status sa_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,

@@ -110,6 +110,18 @@ sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp
 sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
                       int N, int d, float sm_scale, const uint8_t *block_mask, void *stream);
 
+/* Full forward on HOST buffers: q, k, v, o bf16 [B,H,N,d] and block_mask (or NULL) in host
+ * memory, page-locked for the copies to overlap (pageable memory works but serialises).
+ * The B*H heads are independent, so they are processed in chunks of consecutive heads:
+ * the upload of chunk c+1 and the download of chunk c-1 run on two library-owned streams
+ * while chunk c runs sa_attn_fwd's prologue and kernel on `stream`.  The call returns
+ * after enqueueing; the work is complete when `stream` reaches the point after the call
+ * (o is then filled), and q, k, v, o and block_mask must stay valid until then.  Device staging (two chunks) is library-owned, per device and
+ * grow-only, like the workspace.  Calls for the same device from several host threads
+ * are serialised.  Results are identical to sa_attn_fwd on the same inputs. */
+sa_status sa_attn_fwd_host(const void *q, const void *k, const void *v, void *o, int B, int H,
+                           int N, int d, float sm_scale, const uint8_t *block_mask, void *stream);
+
 /* The fused attention kernel alone, on already-quantised inputs (the layouts written by
  * sa_quantize_qk and sa_quantize_v).  For callers that reuse quantised K/V across
  * queries, and for timing the kernel without the prologue.  Allocates nothing. */

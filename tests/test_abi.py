@@ -49,6 +49,8 @@ ODD = ctypes.c_void_p((1 << 20) + 8)  # misaligned
 ])
 def test_attn_fwd_argument_errors(libsa, args, expect):
     assert libsa.raw_library().sa_attn_fwd(*args) == expect
+    # the host-buffer entry point validates the same way before touching CUDA
+    assert libsa.raw_library().sa_attn_fwd_host(*args) == expect
 
 
 def test_other_entry_points_argument_errors(libsa):
