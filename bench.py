@@ -63,14 +63,15 @@ def kernel_source_sha256():
     return h.hexdigest()
 
 
-def recorded_traffic(kernel):
+def recorded_traffic(kernel, workload):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
-    the current kernel sources and for this kernel (else None)."""
+    the current kernel sources, for this kernel and this workload (else None)."""
     p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
     try:
         with open(p) as f:
             rec = json.load(f)
-        if rec.get("kernel_sources_sha256") != kernel_source_sha256() or rec.get("kernel") != kernel:
+        if (rec.get("kernel_sources_sha256") != kernel_source_sha256() or rec.get("kernel") != kernel
+                or rec.get("workload") != workload):
             return None
         return rec
     except Exception:
@@ -301,7 +302,7 @@ def main():
     peak, peak_src = measured_peak()
     achieved = ops_rank / t_attn / 1e12
     kernel = "attn_fwd_kernel" if w.mask_density is not None else "attn_pairs_kernel"
-    traffic = recorded_traffic(kernel)
+    traffic = recorded_traffic(kernel, w.name)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

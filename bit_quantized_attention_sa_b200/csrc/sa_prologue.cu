@@ -87,18 +87,25 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-__device__ __forceinline__ int8_t int8_code(float x, float s)
+// INT8 code of x under scale s: round-half-even of the IEEE quotient x/s, clamped to
+// [-127, 127].  r = 1/s (correctly rounded).  Fast path: y = x*r differs from the IEEE
+// quotient fl(x/s) by at most |x/s| * 3 * 2^-24 < 2.3e-5 (|x/s| <= 127 + tiny), so when y
+// is at least 2^-14 away from every half-integer both round to the same integer; the
+// rare y within 2^-14 of a half-integer takes the exact division.
+__device__ __forceinline__ int int8_code(float x, float s, float r)
 {
     if (s == 0.0f) return 0;
-    int r = __float2int_rn(__fdiv_rn(x, s));
-    r = max(-127, min(127, r));
-    return int8_t(r);
+    const float y = __fmul_rn(x, r);
+    float n = rintf(y);
+    if (fabsf(fabsf(__fsub_rn(y, n)) - 0.5f) < 6.103515625e-05f) n = rintf(__fdiv_rn(x, s));
+    return max(-127, min(127, int(n)));
 }
 
 // One quantisation block of ROWS tokens x 128 channels starting at token r0.
 // mean != nullptr: smooth first (x - mean[c], one fp32 subtraction).  Rows >= N are
 // excluded from the max and stored as zero codes.  scale_out may be null (padding-only
-// block).
+// block).  The block is held as raw bf16 (4 registers per 8 values) and unpacked twice,
+// which keeps the kernel at 4 CTAs per SM.
 template <int ROWS>
 __device__ __forceinline__ void quant_block(const uint16_t *__restrict__ src, int N, int r0,
                                             const float *__restrict__ mean,
@@ -107,26 +114,24 @@ __device__ __forceinline__ void quant_block(const uint16_t *__restrict__ src, in
 {
     constexpr int PER = ROWS * 16 / kThreads;  // 16-byte chunks per thread
     const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
-    float x[PER][8];
+    uint4 raw[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int t = r0 + rs + 16 * i;
+        raw[i] = t < N ? __ldg(reinterpret_cast<const uint4 *>(src + int64_t(t) * kD + cg * 8))
+                       : make_uint4(0, 0, 0, 0);
+    }
     float mc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) mc[e] = mean ? mean[cg * 8 + e] : 0.0f;
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        const int t = r0 + rs + 16 * i;
-        if (t < N) {
-            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src + int64_t(t) * kD + cg * 8));
-            unpack8(u, x[i]);
-            if (mean) {
+        if (r0 + rs + 16 * i < N) {
+            float x[8];
+            unpack8(raw[i], x);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) x[i][e] = __fsub_rn(x[i][e], mc[e]);
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[i][e]));
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[i][e] = 0.0f;
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(mean ? __fsub_rn(x[e], mc[e]) : x[e]));
         }
     }
     amax = warp_max(amax);
@@ -136,22 +141,29 @@ __device__ __forceinline__ void quant_block(const uint16_t *__restrict__ src, in
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w) amax = fmaxf(amax, red[w]);
     const float s = __fdiv_rn(amax, 127.0f);
+    const float r = s == 0.0f ? 0.0f : __frcp_rn(s);
     if (tid == 0 && scale_out) *scale_out = s;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
         const int t = r0 + rs + 16 * i;
         uint32_t lo = 0, hi = 0;
+        if (t < N) {
+            float x[8];
+            unpack8(raw[i], x);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) lo |= uint32_t(uint8_t(int8_code(x[i][e], s))) << (8 * e);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hi |= uint32_t(uint8_t(int8_code(x[i][4 + e], s))) << (8 * e);
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t code = uint32_t(uint8_t(int8_code(mean ? __fsub_rn(x[e], mc[e]) : x[e], s, r)));
+                if (e < 4) lo |= code << (8 * e);
+                else hi |= code << (8 * (e - 4));
+            }
+        }
         *reinterpret_cast<uint2 *>(dst + int64_t(t) * kD + cg * 8) = make_uint2(lo, hi);
     }
 }
 
 // grid (nq + Npad/64, BH): x < nq quantises Q block x; otherwise K block x - nq
 // (blocks at or past nk only zero-fill the padded key rows).
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)
     qk_quant_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, int N,
                     int Npad, int nq, int nk, const float *__restrict__ kmean,
                     int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
@@ -205,14 +217,16 @@ __global__ void __launch_bounds__(kThreads) v_amax_kernel(const uint16_t *__rest
 
 // grid (Npad/128, BH): a 128-token x 128-channel tile, quantised and transposed through
 // shared memory so that both the bf16 reads and the channel-major FP8 writes are
-// coalesced 16-byte accesses.
+// coalesced 16-byte accesses.  The tile is channel-major, 128 B per channel; byte (c, r)
+// sits in 16-byte chunk (r / 16) ^ (g & 7) and 4-byte word ((r % 16) / 4) ^ (g >> 3) of
+// row c, g = c / 8: the 16 threads of a half-warp, each writing one byte for its own group
+// of 8 channels, then hit 16 different banks, and a thread still reads a whole chunk.
 __global__ void __launch_bounds__(kThreads)
     v_quant_kernel(const uint16_t *__restrict__ v, int N, int Npad,
                    const uint32_t *__restrict__ amax_bits, uint8_t *__restrict__ v_t,
                    float *__restrict__ v_scale)
 {
-    constexpr int kPitch = 144;  // bytes per channel row in shared memory (16-B multiple)
-    __shared__ __align__(16) uint8_t tile[kD][kPitch];
+    __shared__ __align__(16) uint8_t tile[kD][kQBlk];
     __shared__ float sv[kD];
     const int64_t bh = blockIdx.y;
     const int t0 = blockIdx.x * kQBlk;
@@ -224,6 +238,7 @@ __global__ void __launch_bounds__(kThreads)
     }
     __syncthreads();
     const uint16_t *vh = v + bh * int64_t(N) * kD;
+    const int swz_chunk = cg & 7, swz_word = cg >> 3;
 #pragma unroll
     for (int i = 0; i < kQBlk * 16 / kThreads; ++i) {
         const int r = rs + 16 * i;
@@ -236,14 +251,15 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
             for (int e = 0; e < 8; ++e) x[e] = 0.0f;
         }
+        const int pos = (((r >> 4) ^ swz_chunk) << 4) | ((((r & 15) >> 2) ^ swz_word) << 2) | (r & 3);
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
             const float s0 = sv[cg * 8 + e], s1 = sv[cg * 8 + e + 1];
             const float y0 = s0 == 0.0f ? 0.0f : __fdiv_rn(x[e], s0);
             const float y1 = s1 == 0.0f ? 0.0f : __fdiv_rn(x[e + 1], s1);
             const uint32_t p = pack_e4m3x2(y0, y1);
-            tile[cg * 8 + e][r] = uint8_t(p & 0xFFu);
-            tile[cg * 8 + e + 1][r] = uint8_t(p >> 8);
+            tile[cg * 8 + e][pos] = uint8_t(p & 0xFFu);
+            tile[cg * 8 + e + 1][pos] = uint8_t(p >> 8);
         }
     }
     __syncthreads();
@@ -251,8 +267,9 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int i = 0; i < kD * 8 / kThreads; ++i) {
         const int qd = tid + kThreads * i;
-        const int c = qd >> 3, part = qd & 7;
-        const uint4 u = *reinterpret_cast<const uint4 *>(&tile[c][part * 16]);
+        const int c = qd >> 3, part = qd & 7, g = c >> 3;
+        const uint4 w = *reinterpret_cast<const uint4 *>(&tile[c][(part ^ (g & 7)) << 4]);
+        const uint4 u = (g >> 3) ? make_uint4(w.y, w.x, w.w, w.z) : w;  // undo the word swizzle
         *reinterpret_cast<uint4 *>(vt + int64_t(c) * Npad + t0 + part * 16) = u;
     }
 }
