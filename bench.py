@@ -78,6 +78,33 @@ def recorded_traffic(kernel, workload):
         return None
 
 
+# ------------------------------------------------------------------------ ranks
+
+
+def rank_workload(w, rank: int):
+    """The workload a rank runs: rank 0 the named one, every other rank the same shapes
+    with its own seed (replicas of independent heads, no data exchanged)."""
+    if rank == 0:
+        return w
+    return type(w)(w.name, w.B, w.H, w.N, w.d, w.outliers, w.mask_density, w.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of the ranks' values (the job takes as long as its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_rank: float, world: int, t_max: float) -> float:
+    """Throughput of the whole job: every rank's work over the slowest rank's time."""
+    return ops_per_rank * world / t_max / 1e12
+
+
 class ClockSampler:
     """nvidia-smi clock/throttle sampling during the timed region."""
 
@@ -216,8 +243,7 @@ def main():
     from bit_quantized_attention_sa_b200 import binding as sa
 
     # each rank owns one replica of the workload (its own seed)
-    q, k, v, m = make_workload(w) if rank == 0 else make_workload(
-        type(w)(w.name, w.B, w.H, w.N, w.d, w.outliers, w.mask_density, w.seed + 7919 * rank))
+    q, k, v, m = make_workload(rank_workload(w, rank))
     shape = (w.B, w.H, w.N, w.d)
 
     def pinned_bf16(a):
@@ -236,12 +262,8 @@ def main():
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     def step():
         sa.sa_attn_fwd(dq, dk, dv, w.sm_scale, block_mask=dm, out=do)
@@ -261,7 +283,7 @@ def main():
     e1.record(stream)
     barrier()
     clocks = sampler.stop()
-    t_step = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.steps)
+    t_step = slowest(e0.elapsed_time(e1) / 1e3 / args.steps)
     assert sa.sa_get_device_status() == 0
 
     # ---- the attention kernel alone (dominant kernel): per-launch duration
@@ -276,7 +298,7 @@ def main():
         sa.sa_attn_fwd_quantized(q8, sq, k8, sk, vt, sv, w.N, w.sm_scale, dm, out=do)
     a1.record(stream)
     barrier()
-    t_attn = max_over_ranks(a0.elapsed_time(a1) / 1e3 / args.steps)
+    t_attn = slowest(a0.elapsed_time(a1) / 1e3 / args.steps)
     del q8, k8, vt
 
     # ---- end to end through the public API with host buffers: sa_attn_fwd_host uploads
@@ -295,10 +317,10 @@ def main():
         sa.sa_attn_fwd_host(hq, hk, hv, out=ho, sm_scale=w.sm_scale, block_mask=hm, stream=stream)
     b1.record(stream)
     barrier()
-    t_e2e = max_over_ranks(b0.elapsed_time(b1) / 1e3 / e2e_steps)
+    t_e2e = slowest(b0.elapsed_time(b1) / 1e3 / e2e_steps)
 
     ops_rank = w.dense_ops
-    value = ops_rank * world / t_step / 1e12
+    value = whole_job_tops(ops_rank, world, t_step)
     peak, peak_src = measured_peak()
     achieved = ops_rank / t_attn / 1e12
     kernel = "attn_fwd_kernel" if w.mask_density is not None else "attn_pairs_kernel"
@@ -328,7 +350,7 @@ def main():
                          "ms_per_launch": t_attn * 1e3,
                          "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
             "cpu_baseline": cpu,
-            "e2e": {"value": ops_rank * world / t_e2e / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_tops(ops_rank, world, t_e2e), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": t_e2e * 1e3},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
