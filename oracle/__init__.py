@@ -59,6 +59,12 @@ def _load():
         lib.sa_oracle_exact_rows.restype = None
         lib.sa_oracle_qk_s32_rows.argtypes = [P, P, I, I, I, I, P, I64, P]
         lib.sa_oracle_qk_s32_rows.restype = None
+        lib.sa_oracle_pool.argtypes = [P, I, I, I, I, I, P]
+        lib.sa_oracle_pool.restype = I
+        lib.sa_oracle_block_scores.argtypes = [P, P, I64, I, I, I, P]
+        lib.sa_oracle_block_scores.restype = None
+        lib.sa_oracle_block_mask.argtypes = [P, I64, I, I, I, I, P]
+        lib.sa_oracle_block_mask.restype = None
         _lib = lib
     return _lib
 
@@ -155,3 +161,41 @@ def qk_s32_rows(q_i8: np.ndarray, k_i8: np.ndarray, N: int, rows) -> np.ndarray:
     _load().sa_oracle_qk_s32_rows(_ptr(q_i8), _ptr(k_i8), B, H, N, d, _ptr(rows),
                                   rows.shape[0], _ptr(out))
     return out
+
+
+def pool(x: np.ndarray, blk: int):
+    """Block means of bf16 bits x [B,H,N,d] over `blk`-token blocks: (fp32
+    [B,H,ceil(N/blk),d], all_sums_exact)."""
+    assert x.dtype == np.uint16
+    B, H, N, d = x.shape
+    out = np.empty((B, H, -(-N // blk), d), np.float32)
+    exact = _load().sa_oracle_pool(_ptr(np.ascontiguousarray(x)), B, H, N, d, int(blk), _ptr(out))
+    return out, bool(exact)
+
+
+def block_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
+    """fp64 pooled scores [B,H,nq,nk] from block means qbar [B,H,nq,d], kbar [B,H,nk,d]."""
+    B, H, nq, d = qbar.shape
+    nk = kbar.shape[2]
+    out = np.empty((B, H, nq, nk), np.float64)
+    _load().sa_oracle_block_scores(_ptr(np.ascontiguousarray(qbar, np.float32)),
+                                   _ptr(np.ascontiguousarray(kbar, np.float32)), B * H, nq, nk,
+                                   d, _ptr(out))
+    return out
+
+
+def mask_from_scores(scores: np.ndarray, keep_per_row: int, keep_diagonal: bool = False) -> np.ndarray:
+    """uint8 keep mask [B,H,nq,nk] from pooled scores (top keep_per_row per row)."""
+    B, H, nq, nk = scores.shape
+    out = np.empty((B, H, nq, nk), np.uint8)
+    _load().sa_oracle_block_mask(_ptr(np.ascontiguousarray(scores, np.float64)), B * H, nq, nk,
+                                 int(keep_per_row), int(bool(keep_diagonal)), _ptr(out))
+    return out
+
+
+def block_mask(q: np.ndarray, k: np.ndarray, keep_per_row: int, keep_diagonal: bool = False):
+    """The whole selector: (mask uint8 [B,H,nq,nk], qbar, kbar, scores, pools_exact)."""
+    qbar, ex_q = pool(q, QBLK)
+    kbar, ex_k = pool(k, KBLK)
+    scores = block_scores(qbar, kbar)
+    return mask_from_scores(scores, keep_per_row, keep_diagonal), qbar, kbar, scores, ex_q and ex_k

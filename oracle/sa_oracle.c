@@ -39,7 +39,10 @@
  * a library cast; quantiser closed forms (exact-integer case, tie cases, block
  * boundaries, shift invariance); attention closed forms (N = 1, identical keys,
  * dominant key), invariants (rows sum to one, constant V columns), brute force against
- * the fp64 exact attention below.
+ * the fp64 exact attention below.  Block-mask producer (end of file): block means against
+ * numpy, pooled scores against an fp64 einsum, the selection rule against an independent
+ * stable sort (ties included), invariants (scaling Q, swapping key blocks) and a planted
+ * key block (tests/test_oracle_mask.py).
  */
 #include <fenv.h>
 #include <math.h>
@@ -399,4 +402,100 @@ void sa_oracle_qk_s32_rows(const int8_t *q_i8, const int8_t *k_i8, int B, int H,
             out[n * Npad + t] = S;
         }
     }
+}
+
+/* ------------------------------------------------------------------------------------
+ * Block-mask producer: the selector ahead of the block skip.
+ *
+ * Sources: NetEase article on the TurboDiffusion release, attention-acceleration section,
+ * SLA figure caption (the attention weights fall into three classes that are computed at
+ * different costs; SLA's forward works from predicted, compressed attention weights);
+ * "Video-Generation-101 research log" section 5.5 table, SpargeAttention row (a two-level
+ * online filter selects blocks ahead of a sparse, low-bit kernel); "Video-Generation-101:
+ * inference systems", kernel paragraph (selector, sparse layout and low-bit kernel are
+ * designed together).
+ * reading: the compressed weights are those of Q mean-pooled per 128-token block against
+ * K mean-pooled per 64-token block (the geometry of the keep mask); a mask row keeps its
+ * keep_per_row highest-scoring key blocks, ties going to the lower block index; the row
+ * softmax and sm_scale are increasing in the score and leave the choice unchanged, so
+ * the raw pooled dot product ranks; optionally the diagonal blocks 2i and 2i+1 (the key
+ * blocks covering the query block's own tokens) are kept as well.
+ * ------------------------------------------------------------------------------------ */
+
+/*
+ * Block means of x (bf16 bits [B,H,N,d]) over blocks of `blk` tokens: out fp32
+ * [B,H,ceil(N/blk),d] = (float)((sum over the block's tokens t < N, t ascending, of
+ * (double)x[t,c]) / (double)count).  Returns 1 if every fp64 sum was exact (TwoSum error
+ * zero), else 0: the sums are then order-independent.
+ */
+int sa_oracle_pool(const uint16_t *x, int B, int H, int N, int d, int blk, float *out)
+{
+    const int64_t BH = (int64_t)B * H, nb = cdiv64(N, blk);
+    int exact = 1;
+    for (int64_t bh = 0; bh < BH; ++bh) {
+        const uint16_t *xh = x + bh * (int64_t)N * d;
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t t0 = b * blk, t1 = (t0 + blk < N) ? t0 + blk : N;
+            for (int c = 0; c < d; ++c) {
+                double s = 0.0, err = 0.0;
+                for (int64_t t = t0; t < t1; ++t) {
+                    const double v = (double)bf16_to_f32(xh[t * d + c]);
+                    const double ns = s + v;
+                    /* TwoSum: err is the exact rounding error of s + v */
+                    const double bv = ns - s, av = ns - bv;
+                    err += (s - av) + (v - bv);
+                    s = ns;
+                }
+                if (err != 0.0) exact = 0;
+                out[(bh * nb + b) * d + c] = (float)(s / (double)(t1 - t0));
+            }
+        }
+    }
+    return exact;
+}
+
+/*
+ * Pooled scores: scores fp64 [BH, nq, nk] = sum over c ascending of
+ * (double)qbar[i,c] * (double)kbar[j,c] (each product exact, one rounding per addition).
+ */
+void sa_oracle_block_scores(const float *qbar, const float *kbar, int64_t BH, int nq, int nk,
+                            int d, double *scores)
+{
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < nq; ++i)
+            for (int j = 0; j < nk; ++j) {
+                const float *a = qbar + (bh * nq + i) * d, *b = kbar + (bh * nk + j) * d;
+                double s = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    const double p = (double)a[c] * (double)b[c];
+                    s = s + p;
+                }
+                scores[(bh * nq + i) * nk + j] = s;
+            }
+}
+
+/*
+ * Keep mask uint8 [BH, nq, nk] from the scores: block j of row i is kept when fewer than
+ * keep_per_row blocks rank before it, where j' ranks before j if its score is larger, or
+ * equal with j' < j; with keep_diagonal the blocks 2i and 2i+1 (when they exist) are kept
+ * too.
+ */
+void sa_oracle_block_mask(const double *scores, int64_t BH, int nq, int nk, int keep_per_row,
+                          int keep_diagonal, uint8_t *mask)
+{
+    for (int64_t bh = 0; bh < BH; ++bh)
+        for (int i = 0; i < nq; ++i) {
+            const double *s = scores + (bh * nq + i) * nk;
+            uint8_t *m = mask + (bh * nq + i) * nk;
+            for (int j = 0; j < nk; ++j) {
+                int rank = 0;
+                for (int jj = 0; jj < nk; ++jj)
+                    if (s[jj] > s[j] || (s[jj] == s[j] && jj < j)) ++rank;
+                m[j] = rank < keep_per_row ? 1 : 0;
+            }
+            if (keep_diagonal) {
+                if (2 * i < nk) m[2 * i] = 1;
+                if (2 * i + 1 < nk) m[2 * i + 1] = 1;
+            }
+        }
 }
