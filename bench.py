@@ -319,6 +319,26 @@ def main():
     barrier()
     t_e2e = slowest(b0.elapsed_time(b1) / 1e3 / e2e_steps)
 
+    # ---- the block-mask producer (selector), timed on its own for masked workloads: it
+    # would run ahead of a masked forward; keep_per_row matches the workload's density
+    selector = None
+    if dm is not None:
+        nk = -(-w.N // 64)
+        keep = max(1, round(w.mask_density * nk))
+        sel = torch.empty_like(dm)
+        for _ in range(args.warmup):
+            sa.sa_block_mask(dq, dk, keep, True, out=sel)
+        barrier()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            sa.sa_block_mask(dq, dk, keep, True, out=sel)
+        s1.record(stream)
+        barrier()
+        selector = {"ms": slowest(s0.elapsed_time(s1) / args.steps), "keep_per_row": keep,
+                    "keep_diagonal": True, "kept_fraction": float(sel.float().mean().item())}
+        del sel
+
     ops_rank = w.dense_ops
     value = whole_job_tops(ops_rank, world, t_step)
     peak, peak_src = measured_peak()
@@ -361,6 +381,7 @@ def main():
             exe = 4.0 * w.d * 128 * 64 * kept
             line["config"]["mask_kept_fraction"] = kept / m.size
             line["executed_tflops"] = exe / t_step / 1e12 * world
+            line["selector"] = selector
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

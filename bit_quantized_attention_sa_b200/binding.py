@@ -32,6 +32,8 @@ _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
+_lib.sa_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
+_lib.sa_debug_pool.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_debug_wait_timeout.argtypes = [_I, _P]
 _lib.sa_debug_exp2_poly.argtypes = [_P, _P, _I, _P]
 _lib.sa_get_device_status.argtypes = []
@@ -44,7 +46,7 @@ _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
               "sa_attn_fwd_quantized",
-              "sa_debug_qk_s32", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
+              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
 
@@ -209,6 +211,34 @@ def sa_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v_fp8_t, v_scale, N: int
                                       float(sm_scale), _ptr(m), _stream(q_i8.device)),
            "sa_attn_fwd_quantized")
     return o
+
+
+def sa_block_mask(q, k, keep_per_row: int, keep_diagonal: bool = False, out=None):
+    """Keep mask uint8 [B,H,ceil(N/128),ceil(N/64)] for bf16 [B,H,N,d] CUDA q, k: the
+    keep_per_row best key blocks per query block by pooled score (plus the diagonal)."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    B, H, N, d = _dims(q)
+    if tuple(k.shape) != (B, H, N, d):
+        raise ValueError("q and k shapes differ")
+    shape = (B, H, -(-N // 128), -(-N // 64))
+    m = torch.empty(shape, dtype=torch.uint8, device=q.device) if out is None else out
+    _need(m, torch.uint8, "out")
+    _check(_lib.sa_block_mask(_ptr(q), _ptr(k), B, H, N, d, int(keep_per_row), int(bool(keep_diagonal)),
+                              _ptr(m), _stream(q.device)), "sa_block_mask")
+    return m
+
+
+def sa_debug_pool(q, k):
+    """Block means (qbar fp32 [B,H,ceil(N/128),d], kbar fp32 [B,H,ceil(N/64),d])."""
+    _need(q, torch.bfloat16, "q")
+    _need(k, torch.bfloat16, "k")
+    B, H, N, d = _dims(q)
+    qbar = torch.empty((B, H, -(-N // 128), d), dtype=torch.float32, device=q.device)
+    kbar = torch.empty((B, H, -(-N // 64), d), dtype=torch.float32, device=q.device)
+    _check(_lib.sa_debug_pool(_ptr(q), _ptr(k), B, H, N, d, _ptr(qbar), _ptr(kbar), _stream(q.device)),
+           "sa_debug_pool")
+    return qbar, kbar
 
 
 def sa_debug_qk_s32(q_i8, k_i8, N: int):

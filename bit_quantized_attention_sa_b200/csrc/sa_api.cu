@@ -416,6 +416,42 @@ sa_status sa_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale, const 
                           block_mask, static_cast<cudaStream_t>(stream));
 }
 
+sa_status sa_block_mask(const void *q, const void *k, int B, int H, int N, int d, int keep_per_row,
+                        int keep_diagonal, uint8_t *block_mask, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (keep_per_row < 1) return SA_ERR_INVALID_ARG;
+    if (!q || !k || !block_mask) return SA_ERR_INVALID_ARG;
+    if ((r = check_ptrs({q, k})) != SA_OK) return r;
+    if (s.nk() > kMaskMaxKeyBlocks) return SA_ERR_UNSUPPORTED;
+    if ((r = check_device()) != SA_OK) return r;
+    const size_t qb = align256(size_t(s.BH() * s.nq()) * kD * 4), kb = align256(size_t(s.BH() * s.nk()) * kD * 4);
+    const size_t sb = size_t(s.BH() * s.nq()) * size_t(s.nk()) * 8;
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(qb + kb + sb, &ws)) != SA_OK) return r;
+    float *qbar = reinterpret_cast<float *>(ws), *kbar = reinterpret_cast<float *>(ws + qb);
+    double *scores = reinterpret_cast<double *>(ws + qb + kb);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_pool_qk(q, k, s, qbar, kbar, st) != cudaSuccess) return SA_ERR_CUDA;
+    return launch_block_select(qbar, kbar, scores, s, keep_per_row, keep_diagonal ? 1 : 0, block_mask, st) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+sa_status sa_debug_pool(const void *q, const void *k, int B, int H, int N, int d, float *qbar,
+                        float *kbar, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({q, k, qbar, kbar})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    return launch_pool_qk(q, k, s, qbar, kbar, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK
+                                                                                              : SA_ERR_CUDA;
+}
+
 sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
                           int32_t *s_out, void *stream)
 {

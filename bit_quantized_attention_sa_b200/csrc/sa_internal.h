@@ -50,6 +50,12 @@ cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k
                                 int Npad, int32_t *s_out, cudaStream_t st);
 cudaError_t launch_debug_wait_timeout(int timeout_us, cudaStream_t st);
 cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t st);
+// ---- block-mask producer (sa_mask.cu)
+constexpr int kMaskMaxKeyBlocks = 4096;  // key blocks per mask row the selector sorts in shared memory
+cudaError_t launch_pool_qk(const void *q, const void *k, const Shape &s, float *qbar, float *kbar,
+                           cudaStream_t st);
+cudaError_t launch_block_select(const float *qbar, const float *kbar, double *scores, const Shape &s,
+                                int keep_per_row, int keep_diagonal, uint8_t *mask, cudaStream_t st);
 // Reads and clears the device status word of the current device (synchronous).
 cudaError_t read_and_clear_status(int *status);
 

@@ -130,6 +130,26 @@ sa_status sa_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale, const 
                                 const float *v_scale, void *o, int B, int H, int N, int d,
                                 float sm_scale, const uint8_t *block_mask, void *stream);
 
+/* Block-mask producer: the keep mask block_mask uint8 [B,H,ceil(N/128),ceil(N/64)] (device,
+ * caller-owned, fully written) for q, k bf16 [B,H,N,d] (device).
+ * Sources: NetEase article on the TurboDiffusion release, attention-acceleration section,
+ * SLA figure caption (selection from predicted, compressed attention weights);
+ * "Video-Generation-101 research log" section 5.5, SpargeAttention row (a block selector
+ * ahead of the sparse low-bit kernel).  Reading: Q is mean-pooled per 128-token block and
+ * K per 64-token block (fp64 sums in token order, rounded to fp32); each pair is scored by
+ * the fp64 dot product of the two means (channel order); row i keeps its keep_per_row
+ * highest-scoring key blocks (ties: lower block index), plus blocks 2i and 2i+1 when
+ * keep_diagonal is non-zero.  keep_per_row >= 1 (values >= ceil(N/64) keep every block).
+ * Needs ceil(N/64) <= 4096 (else SA_ERR_UNSUPPORTED).  Uses the library workspace for the
+ * block means and the scores.  The result is a deterministic function of q and k. */
+sa_status sa_block_mask(const void *q, const void *k, int B, int H, int N, int d, int keep_per_row,
+                        int keep_diagonal, uint8_t *block_mask, void *stream);
+
+/* Debug: the block means of sa_block_mask, qbar fp32 [B,H,ceil(N/128),d] and kbar fp32
+ * [B,H,ceil(N/64),d] (device, caller-owned).  Allocates nothing. */
+sa_status sa_debug_pool(const void *q, const void *k, int B, int H, int N, int d, float *qbar,
+                        float *kbar, void *stream);
+
 /* Debug: the int32 S = q_i8 . k_i8^T tiles computed by the same tcgen05 INT8 path the
  * attention kernel uses, stored to s_out int32 [B,H,Npad,Npad] (padded rows/keys
  * included).  For bit-exact checks on small problems only.  Allocates nothing. */

@@ -29,3 +29,12 @@ def sm_scale(d=128):
 # accumulation order): max-abs and cosine
 O_MAX_ABS = 2e-2
 O_MIN_COS = 0.9995
+
+
+def gpu_rows(o: torch.Tensor, rows):
+    """Rows [(bh, r), ...] of a [B,H,N,d] CUDA output as fp32 numpy [len(rows), d]."""
+    B, H, N, d = o.shape
+    flat = o.reshape(B * H, N, d)
+    idx_bh = torch.tensor([r[0] for r in rows], device=o.device)
+    idx_r = torch.tensor([r[1] for r in rows], device=o.device)
+    return to_host_f32(flat[idx_bh, idx_r])

@@ -62,3 +62,8 @@ def test_other_entry_points_argument_errors(libsa):
                                      ctypes.c_float(0.088), None, None) == 1
     assert lib.sa_debug_qk_s32(FAKE, FAKE, 1, 1, -5, 128, FAKE, None) == 1
     assert lib.sa_debug_wait_timeout(0, None) == 1
+    # the selector: keep_per_row >= 1; at most 4096 key blocks per row
+    assert lib.sa_block_mask(FAKE, FAKE, 1, 1, 128, 128, 0, 0, FAKE, None) == 1
+    assert lib.sa_block_mask(FAKE, FAKE, 1, 1, 128, 128, 1, 0, None, None) == 1
+    assert lib.sa_block_mask(FAKE, FAKE, 1, 1, 4096 * 64 + 1, 128, 1, 0, FAKE, None) == 2
+    assert lib.sa_debug_pool(FAKE, FAKE, 1, 1, 128, 128, ODD, FAKE, None) == 3

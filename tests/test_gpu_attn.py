@@ -9,21 +9,13 @@ import torch
 from bit_quantized_attention_sa_b200.workloads import (WORKLOADS, make_inputs, make_workload,
                                                        sample_rows)
 
-from _helpers import O_MAX_ABS, O_MIN_COS, cosine, sm_scale, to_dev_bf16, to_host_f32
+from _helpers import O_MAX_ABS, O_MIN_COS, cosine, gpu_rows, sm_scale, to_dev_bf16, to_host_f32
 
 pytestmark = pytest.mark.gpu
 
 
 def all_rows(B, H, N):
     return [(bh, r) for bh in range(B * H) for r in range(N)]
-
-
-def gpu_rows(o: torch.Tensor, rows):
-    B, H, N, d = o.shape
-    flat = o.reshape(B * H, N, d)
-    idx_bh = torch.tensor([r[0] for r in rows], device=o.device)
-    idx_r = torch.tensor([r[1] for r in rows], device=o.device)
-    return to_host_f32(flat[idx_bh, idx_r])
 
 
 def compare(o_gpu_rows, o_ref, what):
