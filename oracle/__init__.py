@@ -65,6 +65,10 @@ def _load():
         lib.sa_oracle_block_scores.restype = None
         lib.sa_oracle_block_mask.argtypes = [P, I64, I, I, I, I, P]
         lib.sa_oracle_block_mask.restype = None
+        lib.sa_oracle_w8a8_quantize.argtypes = [P, I64, I64, P, P]
+        lib.sa_oracle_w8a8_quantize.restype = None
+        lib.sa_oracle_w8a8_gemm_rows.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+        lib.sa_oracle_w8a8_gemm_rows.restype = None
         _lib = lib
     return _lib
 
@@ -199,3 +203,29 @@ def block_mask(q: np.ndarray, k: np.ndarray, keep_per_row: int, keep_diagonal: b
     kbar, ex_k = pool(k, KBLK)
     scores = block_scores(qbar, kbar)
     return mask_from_scores(scores, keep_per_row, keep_diagonal), qbar, kbar, scores, ex_q and ex_k
+
+
+def w8a8_quantize(x: np.ndarray):
+    """x: bf16 bits [rows, cols].  Returns (codes int8 [rows, Kpad], scales fp32
+    [ceil(rows/128), ceil(cols/128)]), Kpad = 128 * ceil(cols/128)."""
+    assert x.dtype == np.uint16 and x.ndim == 2
+    rows, cols = x.shape
+    cb = -(-cols // 128)
+    codes = np.empty((rows, cb * 128), np.int8)
+    scales = np.empty((-(-rows // 128), cb), np.float32)
+    _load().sa_oracle_w8a8_quantize(_ptr(np.ascontiguousarray(x)), rows, cols, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def w8a8_gemm_rows(xq, wq, K: int, rows) -> np.ndarray:
+    """fp32 accumulator y [len(rows), N] of the W8A8 linear layer for the given rows of x,
+    from w8a8_quantize(x) and w8a8_quantize(w)."""
+    x8, sx = xq
+    w8, sw = wq
+    M, N = x8.shape[0], w8.shape[0]
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    assert rows.size == 0 or (rows.min() >= 0 and rows.max() < M)
+    y = np.empty((rows.size, N), np.float32)
+    _load().sa_oracle_w8a8_gemm_rows(_ptr(x8), _ptr(sx), _ptr(w8), _ptr(sw), M, N, K, _ptr(rows),
+                                     rows.size, _ptr(y))
+    return y

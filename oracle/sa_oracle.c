@@ -42,7 +42,9 @@
  * the fp64 exact attention below.  Block-mask producer (end of file): block means against
  * numpy, pooled scores against an fp64 einsum, the selection rule against an independent
  * stable sort (ties included), invariants (scaling Q, swapping key blocks) and a planted
- * key block (tests/test_oracle_mask.py).
+ * key block (tests/test_oracle_mask.py).  W8A8 linear layer (end of file): quantiser
+ * against a numpy restatement, exact-integer and single-k-block closed forms, zero blocks,
+ * error against the fp64 product (tests/test_oracle_w8a8.py).
  */
 #include <fenv.h>
 #include <math.h>
@@ -498,4 +500,75 @@ void sa_oracle_block_mask(const double *scores, int64_t BH, int nq, int nk, int 
                 if (2 * i + 1 < nk) m[2 * i + 1] = 1;
             }
         }
+}
+
+/* ------------------------------------------------------------------------------------
+ * W8A8 linear layer: INT8 weights and activations with per-128x128-block scales.
+ *
+ * Sources: NetEase article on the TurboDiffusion release, "W8A8 linear-layer
+ * quantisation" section (the weights and activations of the linear layers are quantised to
+ * 8 bits in blocks of 128 x 128 and the products run on INT8 tensor cores); "AIGC weekend
+ * special 5.10" section 1.2 Method item (4) (W8A8: weights and activations of the
+ * non-attention linear layers to INT8).
+ * reading: a block's scale is max|x|/127 over its (valid) elements and its codes are
+ * round-half-even(x/scale) clamped to [-127, 127], as for Q and K above; y = x . w^T for
+ * x [M,K] and w [N,K] (the out x in layout of a linear layer's weight); the int32 product
+ * of one 128-wide k-block is exact and is added to an fp32 accumulator as
+ * acc = fmaf((float)S, sx[m-block, k-block] * sw[n-block, k-block], acc), k-blocks in
+ * ascending order; y is acc rounded to bf16 (nearest-even).  K is padded to a multiple of
+ * 128 with zero codes.
+ * ------------------------------------------------------------------------------------ */
+
+/*
+ * Codes int8 [rows, Kpad] (Kpad = 128 * ceil(cols/128), padding zero) and scales fp32
+ * [ceil(rows/128), ceil(cols/128)] of x (bf16 bits [rows, cols]), per 128 x 128 block.
+ */
+void sa_oracle_w8a8_quantize(const uint16_t *x, int64_t rows, int64_t cols, int8_t *codes,
+                             float *scales)
+{
+    const int64_t rb = cdiv64(rows, 128), cb = cdiv64(cols, 128), kpad = cb * 128;
+    fesetround(FE_TONEAREST);
+    for (int64_t i = 0; i < rows * kpad; ++i) codes[i] = 0;
+    for (int64_t a = 0; a < rb; ++a)
+        for (int64_t b = 0; b < cb; ++b) {
+            const int64_t r0 = a * 128, r1 = r0 + 128 < rows ? r0 + 128 : rows;
+            const int64_t c0 = b * 128, c1 = c0 + 128 < cols ? c0 + 128 : cols;
+            float amax = 0.0f;
+            for (int64_t r = r0; r < r1; ++r)
+                for (int64_t c = c0; c < c1; ++c) {
+                    const float v = fabsf(bf16_to_f32(x[r * cols + c]));
+                    if (v > amax) amax = v;
+                }
+            const float s = amax / 127.0f;
+            scales[a * cb + b] = s;
+            for (int64_t r = r0; r < r1; ++r)
+                for (int64_t c = c0; c < c1; ++c)
+                    codes[r * kpad + c] = int8_code(bf16_to_f32(x[r * cols + c]), s);
+        }
+}
+
+/*
+ * y fp32 [nrows, N] for the given rows of x: y[r, n] = the fp32 accumulator above (before
+ * the bf16 rounding), from codes x8 [M, Kpad], w8 [N, Kpad] and scales sx, sw.
+ */
+void sa_oracle_w8a8_gemm_rows(const int8_t *x8, const float *sx, const int8_t *w8,
+                              const float *sw, int64_t M, int64_t N, int64_t K,
+                              const int64_t *rows, int64_t nrows, float *y)
+{
+    const int64_t cb = cdiv64(K, 128), kpad = cb * 128;
+    (void)M;
+    for (int64_t ri = 0; ri < nrows; ++ri) {
+        const int64_t m = rows[ri];
+        for (int64_t n = 0; n < N; ++n) {
+            float acc = 0.0f;
+            for (int64_t b = 0; b < cb; ++b) {
+                int32_t S = 0;
+                for (int64_t k = b * 128; k < b * 128 + 128; ++k)
+                    S += (int32_t)x8[m * kpad + k] * (int32_t)w8[n * kpad + k];
+                const float s = sx[(m / 128) * cb + b] * sw[(n / 128) * cb + b];
+                acc = fmaf((float)S, s, acc);
+            }
+            y[ri * N + n] = acc;
+        }
+    }
 }
