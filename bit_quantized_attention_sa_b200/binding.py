@@ -34,6 +34,9 @@ _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
 _lib.sa_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
 _lib.sa_debug_pool.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
+_lib.sa_w8a8_quantize.argtypes = [_P, _I, _I, _P, _P, _P]
+_lib.sa_w8a8_gemm.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P, _P]
+_lib.sa_w8a8_linear.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.sa_debug_wait_timeout.argtypes = [_I, _P]
 _lib.sa_debug_exp2_poly.argtypes = [_P, _P, _I, _P]
 _lib.sa_get_device_status.argtypes = []
@@ -46,7 +49,7 @@ _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
               "sa_attn_fwd_quantized",
-              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
+              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
 
@@ -239,6 +242,67 @@ def sa_debug_pool(q, k):
     _check(_lib.sa_debug_pool(_ptr(q), _ptr(k), B, H, N, d, _ptr(qbar), _ptr(kbar), _stream(q.device)),
            "sa_debug_pool")
     return qbar, kbar
+
+
+def _matrix(t: torch.Tensor, name: str):
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor")
+    return int(t.shape[0]), int(t.shape[1])
+
+
+def sa_w8a8_quantize(x: torch.Tensor):
+    """128 x 128 block quantisation of bf16 x [rows, cols]: (codes int8 [rows, kpad],
+    scales fp32 [ceil(rows/128), kpad/128]), kpad = 128 * ceil(cols/128)."""
+    _need(x, torch.bfloat16, "x")
+    rows, cols = _matrix(x, "x")
+    kpad = -(-cols // 128) * 128
+    codes = torch.empty((rows, kpad), dtype=torch.int8, device=x.device)
+    scales = torch.empty((-(-rows // 128), kpad // 128), dtype=torch.float32, device=x.device)
+    _check(_lib.sa_w8a8_quantize(_ptr(x), rows, cols, _ptr(codes), _ptr(scales), _stream(x.device)),
+           "sa_w8a8_quantize")
+    return codes, scales
+
+
+def _w8a8_out(M, N, device, out):
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=device) if out is None else out
+    _need(y, torch.bfloat16, "out")
+    if tuple(y.shape) != (M, N):
+        raise ValueError("out has the wrong shape")
+    return y
+
+
+def sa_w8a8_gemm(xq, wq, K: int, out=None):
+    """bf16 y [M, N] = the block-scaled INT8 product of xq = (codes [M, kpad], scales) and
+    wq = (codes [N, kpad], scales), as returned by sa_w8a8_quantize of x [M, K], w [N, K]."""
+    (xc, xs), (wc, ws) = xq, wq
+    for t, dt, name in ((xc, torch.int8, "x codes"), (xs, torch.float32, "x scales"),
+                        (wc, torch.int8, "w codes"), (ws, torch.float32, "w scales")):
+        _need(t, dt, name)
+    M, kpad = _matrix(xc, "x codes")
+    N, kpad_w = _matrix(wc, "w codes")
+    if kpad != kpad_w or kpad != -(-int(K) // 128) * 128:
+        raise ValueError("codes widths do not match K")
+    y = _w8a8_out(M, N, xc.device, out)
+    _check(_lib.sa_w8a8_gemm(_ptr(xc), _ptr(xs), _ptr(wc), _ptr(ws), M, N, int(K), _ptr(y), _stream(xc.device)),
+           "sa_w8a8_gemm")
+    return y
+
+
+def sa_w8a8_linear(x: torch.Tensor, wq, out=None):
+    """bf16 y [M, N] = W8A8 linear layer of bf16 x [M, K] with the pre-quantised weight
+    wq = (codes [N, kpad], scales) of w [N, K]."""
+    wc, ws = wq
+    _need(x, torch.bfloat16, "x")
+    _need(wc, torch.int8, "w codes")
+    _need(ws, torch.float32, "w scales")
+    M, K = _matrix(x, "x")
+    N, kpad = _matrix(wc, "w codes")
+    if kpad != -(-K // 128) * 128:
+        raise ValueError("w codes width does not match K")
+    y = _w8a8_out(M, N, x.device, out)
+    _check(_lib.sa_w8a8_linear(_ptr(x), _ptr(wc), _ptr(ws), M, N, K, _ptr(y), _stream(x.device)),
+           "sa_w8a8_linear")
+    return y
 
 
 def sa_debug_qk_s32(q_i8, k_i8, N: int):

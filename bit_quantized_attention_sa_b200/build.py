@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsa.so")
-SOURCES = ["sa_api.cu", "sa_prologue.cu", "sa_attn.cu", "sa_mask.cu"]
+SOURCES = ["sa_api.cu", "sa_prologue.cu", "sa_attn.cu", "sa_mask.cu", "sa_w8a8.cu"]
 HEADERS = ["sa_ptx.cuh", "sa_internal.h", "sa_attn_pairs.cuh"]
 
 NVCC_FLAGS = [
@@ -56,7 +56,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
             cmd = [nvcc()] + NVCC_FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", s, "-o", o]
             subprocess.run(cmd, check=True)
     if force or _stale(LIB, objs):
-        cmd = [nvcc(), "-shared", "-cudart", "static", "-o", LIB + ".tmp"] + objs
+        cmd = [nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static", "-o", LIB + ".tmp"] + objs
         subprocess.run(cmd, check=True)
         os.replace(LIB + ".tmp", LIB)
     return LIB

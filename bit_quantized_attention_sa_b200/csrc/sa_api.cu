@@ -452,6 +452,70 @@ sa_status sa_debug_pool(const void *q, const void *k, int B, int H, int N, int d
                                                                                               : SA_ERR_CUDA;
 }
 
+sa_status sa_w8a8_quantize(const void *x, int rows, int cols, int8_t *codes, float *scales, void *stream)
+{
+    if (rows < 1 || cols < 1) return SA_ERR_INVALID_ARG;
+    if (cols % 8 != 0 || cdiv(rows, 128) > 65535) return SA_ERR_UNSUPPORTED;
+    sa_status r = check_ptrs({x, codes, scales});
+    if (r != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    return launch_w8a8_quantize(x, rows, cols, codes, scales, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+static sa_status w8a8_gemm_checked(const int8_t *x_codes, const float *x_scales, const int8_t *w_codes,
+                                   const float *w_scales, int M, int N, int K, void *y, cudaStream_t st)
+{
+    const int64_t kpad = cdiv(K, 128) * 128;
+    CUtensorMap tx, tw;
+    if (!encode_tmap_2d_u8(&tx, x_codes, uint64_t(kpad), uint64_t(M), uint64_t(kpad), 128, kW8a8BoxRows,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tmap_2d_u8(&tw, w_codes, uint64_t(kpad), uint64_t(N), uint64_t(kpad), 128, kW8a8BoxRows,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+        return SA_ERR_CUDA;
+    return launch_w8a8_gemm(tx, tw, x_scales, w_scales, M, N, int(kpad / 128), y, st) == cudaSuccess ? SA_OK
+                                                                                                : SA_ERR_CUDA;
+}
+
+// need_k8: x is quantised here from bf16 rows, read 8 values (16 bytes) at a time
+static sa_status check_w8a8_sizes(int M, int N, int K, bool need_k8)
+{
+    if (M < 1 || N < 1 || K < 1) return SA_ERR_INVALID_ARG;
+    if (N % 8 != 0 || (need_k8 && K % 8 != 0)) return SA_ERR_UNSUPPORTED;
+    // TMA row coordinates and tile counts are 32-bit; grid rows of the quantiser <= 65535
+    if (cdiv(M, 128) > 65535 || cdiv(N, 128) > 65535) return SA_ERR_UNSUPPORTED;
+    return SA_OK;
+}
+
+sa_status sa_w8a8_gemm(const int8_t *x_codes, const float *x_scales, const int8_t *w_codes, const float *w_scales,
+                       int M, int N, int K, void *y, void *stream)
+{
+    sa_status r = check_w8a8_sizes(M, N, K, false);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({x_codes, x_scales, w_codes, w_scales, y})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    return w8a8_gemm_checked(x_codes, x_scales, w_codes, w_scales, M, N, K, y, static_cast<cudaStream_t>(stream));
+}
+
+sa_status sa_w8a8_linear(const void *x, const int8_t *w_codes, const float *w_scales, int M, int N, int K,
+                         void *y, void *stream)
+{
+    sa_status r = check_w8a8_sizes(M, N, K, true);
+    if (r != SA_OK) return r;
+    if ((r = check_ptrs({x, w_codes, w_scales, y})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    const size_t kpad = size_t(cdiv(K, 128)) * 128;
+    const size_t cb = align256(size_t(M) * kpad), sb = size_t(cdiv(M, 128)) * size_t(kpad / 128) * 4;
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(cb + sb, &ws)) != SA_OK) return r;
+    int8_t *xc = reinterpret_cast<int8_t *>(ws);
+    float *xs = reinterpret_cast<float *>(ws + cb);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_w8a8_quantize(x, M, K, xc, xs, st) != cudaSuccess) return SA_ERR_CUDA;
+    return w8a8_gemm_checked(xc, xs, w_codes, w_scales, M, N, K, y, st);
+}
+
 sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
                           int32_t *s_out, void *stream)
 {
@@ -494,9 +558,10 @@ sa_status sa_debug_exp2_poly(const float *x, float *y, int n, void *stream)
 
 sa_status sa_get_device_status(void)
 {
-    int st = 0;
-    if (read_and_clear_status(&st) != cudaSuccess) return SA_ERR_CUDA;
-    return st == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
+    int st = 0, st_w8a8 = 0;
+    if (read_and_clear_status(&st) != cudaSuccess || read_and_clear_w8a8_status(&st_w8a8) != cudaSuccess)
+        return SA_ERR_CUDA;
+    return st == 0 && st_w8a8 == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
 }
 
 const char *sa_status_string(sa_status s)

@@ -56,6 +56,18 @@ cudaError_t launch_pool_qk(const void *q, const void *k, const Shape &s, float *
                            cudaStream_t st);
 cudaError_t launch_block_select(const float *qbar, const float *kbar, double *scores, const Shape &s,
                                 int keep_per_row, int keep_diagonal, uint8_t *mask, cudaStream_t st);
+// ---- W8A8 linear layer (sa_w8a8.cu)
+// x bf16 [rows, cols] (cols % 8 == 0) -> codes int8 [rows, kpad = 128 * ceil(cols / 128)]
+// (padding columns zero) and scales fp32 [ceil(rows / 128), ceil(cols / 128)].
+cudaError_t launch_w8a8_quantize(const void *x, int64_t rows, int64_t cols, int8_t *codes, float *scales,
+                                 cudaStream_t st);
+// y bf16 [M, N] (N % 8 == 0) from the codes behind tm_x ([M, kpad]) and tm_w ([N, kpad]),
+// both encoded with a box of 128 bytes x kW8a8BoxRows rows and 128-byte swizzle, and their
+// block scales, nkb = kpad / 128.
+constexpr int kW8a8BoxRows = 128;
+cudaError_t launch_w8a8_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const float *sx,
+                             const float *sw, int M, int N, int nkb, void *y, cudaStream_t st);
+cudaError_t read_and_clear_w8a8_status(int *status);
 // Reads and clears the device status word of the current device (synchronous).
 cudaError_t read_and_clear_status(int *status);
 

@@ -139,3 +139,52 @@ def sample_rows(B: int, H: int, N: int, per_head: int, seed: int = 7):
             cand.add(int(rng.integers(0, N)))
         rows.extend((bh, r) for r in sorted(cand)[:per_head] if r < N)
     return rows
+
+
+# ---- linear layers (the W8A8 GEMM): activations x [M, K] and weights w [N, K] of the
+# Wan2.1-14B transformer block (hidden 5120, feed-forward 13824) over the latent tokens.
+@dataclass(frozen=True)
+class LinearWorkload:
+    name: str
+    M: int
+    N: int
+    K: int
+    seed: int = 0
+
+    @property
+    def ops(self) -> float:
+        """2*M*N*K: one multiply and one add per term of the product."""
+        return 2.0 * self.M * self.N * self.K
+
+
+LINEAR_WORKLOADS = {
+    "small-m300-n264-k1000": LinearWorkload("small-m300-n264-k1000", 300, 264, 1000, seed=2000),
+    "wan14b-720p-ffn-up-m75600-n13824-k5120": LinearWorkload(
+        "wan14b-720p-ffn-up-m75600-n13824-k5120", 75600, 13824, 5120, seed=2001),
+}
+
+
+def make_linear_inputs(M: int, N: int, K: int, seed: int = 0, outliers: bool = True):
+    """Return (x, w), uint16 bf16 bits [M, K] and [N, K].
+
+    Recipe: one ``Generator(PCG64(seed))`` stream drawn in the order x, w, outlier picks;
+    x ~ N(0, 1) drawn in chunks of 4096 rows (same stream as one draw), w ~ N(0, 1) *
+    K^-1/2; with ``outliers`` round(1% of K) activation channels (at least one), picked by
+    the stream, are multiplied by 8 (the channel outliers of transformer activations);
+    both rounded once from fp32 to bf16."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = np.empty((M, K), np.uint16)
+    chunks = []
+    for r0 in range(0, M, 4096):
+        chunks.append((r0, rng.standard_normal((min(M, r0 + 4096) - r0, K), dtype=np.float32)))
+    w = f32_to_bf16_bits(rng.standard_normal((N, K), dtype=np.float32) * np.float32(1.0 / np.sqrt(K)))
+    cols = rng.choice(K, size=max(1, int(round(0.01 * K))), replace=False) if outliers else []
+    for r0, xf in chunks:
+        if len(cols):
+            xf[:, cols] *= np.float32(8.0)
+        x[r0:r0 + xf.shape[0]] = f32_to_bf16_bits(xf)
+    return x, w
+
+
+def make_linear_workload(w: LinearWorkload):
+    return make_linear_inputs(w.M, w.N, w.K, seed=w.seed)

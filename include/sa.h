@@ -150,6 +150,38 @@ sa_status sa_block_mask(const void *q, const void *k, int B, int H, int N, int d
 sa_status sa_debug_pool(const void *q, const void *k, int B, int H, int N, int d, float *qbar,
                         float *kbar, void *stream);
 
+/* ---- W8A8 linear layer: y = x . w^T with x [M,K] and w [N,K] both quantised to INT8 with
+ * one scale per 128 x 128 block, products on the INT8 tensor cores.
+ * Sources: NetEase article on the TurboDiffusion release, W8A8 linear-layer section
+ * (weights and activations of the linear layers to 8 bits, 128 x 128 blocks, INT8 tensor
+ * cores); "AIGC weekend special 5.10" section 1.2 Method, item (4).
+ * Definition (readings where the pages are silent): a block's scale is max|x| / 127 over
+ * the block (fp32), codes rint_even(x / scale) clamped to [-127, 127], a zero block has
+ * scale 0 and codes 0; K is padded with zero codes to kpad = 128 * ceil(K/128);
+ * y[m,n] = bf16_rn( acc ), acc = 0, then for each k-block b = 0, 1, ... in order:
+ *   acc = fmaf( (float) S_b, sx[m/128][b] * sw[n/128][b], acc )   (fp32, one rounding),
+ * S_b the exact int32 dot product of the 128 codes of block b. */
+
+/* Block quantisation of x bf16 [rows, cols] (device): codes int8 [rows, 128*ceil(cols/128)]
+ * (padding columns written as zero), scales fp32 [ceil(rows/128), ceil(cols/128)] (both
+ * device, caller-owned).  cols % 8 == 0 and ceil(rows/128) <= 65535, else SA_ERR_UNSUPPORTED.
+ * Bit-identical to the definition above.  Allocates nothing.  Used for the weights once and
+ * for the activations on every call. */
+sa_status sa_w8a8_quantize(const void *x, int rows, int cols, int8_t *codes, float *scales, void *stream);
+
+/* y bf16 [M, N] (device, caller-owned) from quantised x (codes [M, kpad], scales
+ * [ceil(M/128), kpad/128]) and w (codes [N, kpad], scales [ceil(N/128), kpad/128]), as laid
+ * out by sa_w8a8_quantize.  N % 8 == 0, else SA_ERR_UNSUPPORTED.
+ * Bit-identical to the definition above.  Allocates nothing. */
+sa_status sa_w8a8_gemm(const int8_t *x_codes, const float *x_scales, const int8_t *w_codes,
+                       const float *w_scales, int M, int N, int K, void *y, void *stream);
+
+/* The linear layer: quantises x bf16 [M, K] into the library workspace, then sa_w8a8_gemm
+ * with the pre-quantised weight.  K % 8 == 0 and N % 8 == 0, else SA_ERR_UNSUPPORTED.
+ * Workspace rules as for sa_attn_fwd. */
+sa_status sa_w8a8_linear(const void *x, const int8_t *w_codes, const float *w_scales, int M, int N,
+                         int K, void *y, void *stream);
+
 /* Debug: the int32 S = q_i8 . k_i8^T tiles computed by the same tcgen05 INT8 path the
  * attention kernel uses, stored to s_out int32 [B,H,Npad,Npad] (padded rows/keys
  * included).  For bit-exact checks on small problems only.  Allocates nothing. */

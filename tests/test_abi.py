@@ -67,3 +67,21 @@ def test_other_entry_points_argument_errors(libsa):
     assert lib.sa_block_mask(FAKE, FAKE, 1, 1, 128, 128, 1, 0, None, None) == 1
     assert lib.sa_block_mask(FAKE, FAKE, 1, 1, 4096 * 64 + 1, 128, 1, 0, FAKE, None) == 2
     assert lib.sa_debug_pool(FAKE, FAKE, 1, 1, 128, 128, ODD, FAKE, None) == 3
+
+
+def test_w8a8_argument_errors(libsa):
+    lib = libsa.raw_library()
+    # quantiser: sizes >= 1, cols a multiple of 8, aligned pointers
+    assert lib.sa_w8a8_quantize(FAKE, 0, 128, FAKE, FAKE, None) == 1
+    assert lib.sa_w8a8_quantize(FAKE, 128, 100, FAKE, FAKE, None) == 2
+    assert lib.sa_w8a8_quantize(FAKE, 128, 128, ODD, FAKE, None) == 3
+    assert lib.sa_w8a8_quantize(None, 128, 128, FAKE, FAKE, None) == 1
+    # GEMM: M, N, K >= 1; N a multiple of 8 (K is free: the codes are padded to 128)
+    assert lib.sa_w8a8_gemm(FAKE, FAKE, FAKE, FAKE, 128, 0, 128, FAKE, None) == 1
+    assert lib.sa_w8a8_gemm(FAKE, FAKE, FAKE, FAKE, 128, 100, 128, FAKE, None) == 2
+    assert lib.sa_w8a8_gemm(FAKE, FAKE, FAKE, None, 128, 128, 128, FAKE, None) == 1
+    assert lib.sa_w8a8_gemm(FAKE, FAKE, FAKE, FAKE, 128, 128, 128, ODD, None) == 3
+    assert lib.sa_w8a8_linear(FAKE, FAKE, FAKE, -1, 128, 128, FAKE, None) == 1
+    assert lib.sa_w8a8_linear(FAKE, FAKE, FAKE, 128, 12, 128, FAKE, None) == 2
+    assert lib.sa_w8a8_linear(FAKE, FAKE, FAKE, 128, 128, 100, FAKE, None) == 2
+    assert lib.sa_w8a8_linear(ODD, FAKE, FAKE, 128, 128, 128, FAKE, None) == 3
