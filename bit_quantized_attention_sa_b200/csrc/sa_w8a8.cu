@@ -21,16 +21,17 @@
 //   warp 8      producer (both CTAs): TMA loads of this CTA's x half (128 rows x 128 B)
 //               and w half (128 rows x 128 B) of each k-block into a 6-stage ring; both
 //               halves complete on the full barrier of CTA 0.
-//   warp 9      MMA issuer (one thread of CTA 0): 4 MMAs per k-block into one of two
-//               int32 accumulators (256 columns each), committed to the stage's empty
-//               barrier and the accumulator's full barrier in both CTAs.
+//   warps 9-10  MMA issuers (lane 0 of each, in CTA 0): warp 9 takes the even k-blocks
+//               and warp 10 the odd ones, each into its own int32 accumulator (256
+//               columns), 4 MMAs per k-block, committed to the stage's empty barrier and
+//               the accumulator's full barrier in both CTAs.  Two issuing threads keep
+//               the tensor pipe fed where one thread's issue rate falls short.
 //   warps 0-7   epilogue (both CTAs): warp w owns TMEM lane quarter w % 4 and columns
 //               128 * (w / 4) .. +127 (one weight block); per k-block it reads its int32
-//               block, releases the accumulator (to CTA 0's empty barrier) and folds the
-//               block into 128 fp32 registers with the block's scale; after the last
-//               k-block it stores bf16 rows.
-//   warps 10-11 idle (complete the third warpgroup for the register split: the epilogue
-//               raises its registers to 232, the rest lower theirs to 40).
+//               block 16 columns at a time, the next load in flight while the previous
+//               16 columns are converted and folded into 128 fp32 registers with the
+//               block's scale, releases the accumulator (to CTA 0's empty barrier) as soon
+//               as the last load has landed, and after the last k-block stores bf16 rows.
 // Every mbarrier wait is bounded (sa_ptx.cuh); on expiry the kernel records the device
 // timeout status and exits.
 #include <cstdint>
@@ -45,10 +46,10 @@ __device__ int g_w8a8_status;  // 0 = OK, 6 = a bounded wait expired
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 352;  // 8 epilogue warps, the producer and two MMA issuers
 constexpr int kStages = 6;
 constexpr int kPairM = 256, kTileN = 256, kKB = 128, kHalf = 128;
-constexpr int kWarpProducer = 8, kWarpMma = 9;
+constexpr int kWarpProducer = 8, kWarpMma = 9, kNumIssuers = 2;
 constexpr uint32_t kHalfTileBytes = kHalf * kKB;              // 16 KB: 128 rows of one k-block
 static_assert(kW8a8BoxRows == kHalf, "each TMA load fills one half tile");
 constexpr uint32_t kStageBytes = 2 * kHalfTileBytes;           // this CTA's x half + w half
@@ -58,25 +59,11 @@ constexpr int kBarFull = 0, kBarEmpty = kStages, kBarAccFull = 2 * kStages, kBar
 constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
 constexpr uint32_t kSmemAlloc = kOffMisc + 16 + 1024;
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory per CTA");
-constexpr int kLaunchRegs = (65536 / kThreads) / 8 * 8;
-constexpr int kRegsEpi = 232, kRegsCtrl = 40;
-static_assert(128 * (2 * kRegsEpi + kRegsCtrl) <= kLaunchRegs * kThreads, "register split");
 constexpr uint32_t kIdesc = idesc_s8_s32(kPairM, kTileN);
 constexpr int kEpilogueWarps = 8;
+static_assert(kStages % kNumIssuers == 0, "each stage is always consumed by the same issuer");
 
 __device__ __forceinline__ void record_timeout() { atomicExch(&g_w8a8_status, int(6)); }
-
-template <uint32_t NR>
-__device__ __forceinline__ void setmaxnreg_inc()
-{
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(NR));
-}
-
-template <uint32_t NR>
-__device__ __forceinline__ void setmaxnreg_dec()
-{
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(NR));
-}
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
@@ -144,19 +131,6 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-// Exact int32 -> fp32 of a block sum.  A 128-term sum of products of 8-bit codes has
-// |S| <= 128 * 128 * 128 = 2^21 < 2^22, so the bit pattern of 1.5 * 2^23 plus S is the
-// float 1.5 * 2^23 + S (unit spacing there), and subtracting 1.5 * 2^23 leaves S exactly;
-// an integer add and a packed subtract in place of two slower conversions.
-__device__ __forceinline__ void int32_pair_to_f32(uint32_t a, uint32_t b, float &fa, float &fb)
-{
-    constexpr uint32_t kMagicBits = 0x4B400000u;  // 1.5 * 2^23
-    constexpr float kMagic = 12582912.0f;
-    fma2(fa, fb, __uint_as_float(a + kMagicBits), __uint_as_float(b + kMagicBits), 1.0f, 1.0f, -kMagic,
-         -kMagic);
-}
-
-
 // ------------------------------------------------------------------ CTA-pair primitives
 // (cluster of two CTAs; every tcgen05 instruction of the kernel uses cta_group::2)
 
@@ -187,6 +161,32 @@ __device__ __forceinline__ uint32_t cluster_addr(uint32_t addr, uint32_t rank)
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t caddr)
 {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+
+// 16 columns of this warp's TMEM lanes, without waiting: the registers are valid only
+// after tmem_wait_ld() and regs_ready16().
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Makes the compiler treat r as produced here, after the wait, so no use of the loaded
+// values is scheduled before it.
+__device__ __forceinline__ void regs_ready16(uint32_t (&r)[16])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
 }
 
 // 2-D tiled TMA load into this CTA's shared memory whose byte count completes on the
@@ -284,7 +284,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (warp >= kWarpProducer) {
-        setmaxnreg_dec<kRegsCtrl>();
         if (warp == kWarpProducer && lane == 0) {
             prefetch_tmap(&tm_x);
             prefetch_tmap(&tm_w);
@@ -308,11 +307,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (uint32_t d = g > kStages ? g - kStages : 0; d < g && ok; ++d)
                 ok = mbar_wait(bar(kBarEmpty + d % kStages), (d / kStages) & 1, abort_flag);
             if (!ok) { *abort_flag = 1; record_timeout(); }
-        } else if (warp == kWarpMma && lane == 0 && rank == 0) {
+        } else if (warp >= kWarpMma && warp < kWarpMma + kNumIssuers && lane == 0 && rank == 0) {
             bool ok = true;
             uint32_t g = 0;
+            const uint32_t me = uint32_t(warp - kWarpMma);  // this issuer's k-blocks: g % 2 == me
             for (int t = pair; t < ntiles && ok; t += npairs) {
                 for (int b = 0; b < nkb && ok; ++b, ++g) {
+                    if ((g & 1) != me) continue;
                     const uint32_t st = g % kStages, ab = g & 1;
                     ok = mbar_wait(bar(kBarFull + st), (g / kStages) & 1, abort_flag);
                     if (ok && g >= 2) ok = mbar_wait(bar(kBarAccEmpty + ab), ((g >> 1) - 1) & 1, abort_flag);
@@ -333,7 +334,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue warps 0-7
-        setmaxnreg_inc<kRegsEpi>();
         const int wq = warp & 3, half = warp >> 2;
         const uint32_t lane_addr = uint32_t(wq * 32) << 16;
         const int nbm = (M + kHalf - 1) / kHalf, nbn = (N + kHalf - 1) / kHalf;
@@ -354,24 +354,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 if (ok) tc_fence_after();
                 const uint32_t ta = tmem + lane_addr + ab * kTileN + half * 128;
+                // 16-column chunks: chunk q + 1 is loading while chunk q is folded in
+                uint32_t va[16], vb[16];
+                if (ok) tmem_ld16_nowait(ta, va);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    uint32_t v[16];
-                    if (ok) tmem_ld16_wait(ta + 16 * q, v);
+                    uint32_t(&cur)[16] = (q & 1) ? vb : va;
+                    uint32_t(&nxt)[16] = (q & 1) ? va : vb;
+                    if (ok) {
+                        tmem_wait_ld();
+                        regs_ready16(cur);
+                    }
                     if (q == 7) {
                         // the warp's whole block is in registers: release the accumulator
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster_relaxed(cluster_addr(bar(kBarAccEmpty + ab), 0));
+                    } else if (ok) {
+                        tmem_ld16_nowait(ta + 16 * (q + 1), nxt);
                     }
                     if (ok) {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 2) {
-                            float f0, f1;
-                            int32_pair_to_f32(v[i], v[i + 1], f0, f1);
-                            fma2(acc[16 * q + i], acc[16 * q + i + 1], f0, f1, s, s, acc[16 * q + i],
-                                 acc[16 * q + i + 1]);
-                        }
+                        for (int i = 0; i < 16; i += 2)
+                            fma2(acc[16 * q + i], acc[16 * q + i + 1], __int2float_rn(int(cur[i])),
+                                 __int2float_rn(int(cur[i + 1])), s, s, acc[16 * q + i], acc[16 * q + i + 1]);
                     }
                 }
             }
