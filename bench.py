@@ -27,10 +27,12 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from bit_quantized_attention_sa_b200.workloads import WORKLOADS, make_workload  # noqa: E402
+from bit_quantized_attention_sa_b200.workloads import (LINEAR_WORKLOADS, WORKLOADS, make_linear_workload,  # noqa: E402
+                                                       make_workload)
 
 METRIC = "quantized attention TOPS (4·H·N²·d/s) and % of B200 dense INT8/FP8 peak"
 DEFAULT_WORKLOAD = "wan14b-720p-h40-n75600"
+DEFAULT_LINEAR = "wan14b-720p-ffn-up-m75600-n13824-k5120"
 DATASHEET_TOPS = 4500.0  # B200 dense INT8 / FP8 tensor peak (NVIDIA datasheet)
 KERNELS_PER_STEP = 6      # k_partial, k_mean, qk_quant, v_amax, v_quant, attn_fwd
 
@@ -222,6 +224,8 @@ def main():
     ap.add_argument("--oracle-rows", type=int, default=64,
                     help="query rows in the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--linear-workload", default=DEFAULT_LINEAR, choices=list(LINEAR_WORKLOADS) + ["none"],
+                    help="W8A8 linear layer timed beside the attention step ('none' skips it)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = WORKLOADS[args.workload]
@@ -339,9 +343,48 @@ def main():
                     "keep_diagonal": True, "kept_fraction": float(sel.float().mean().item())}
         del sel
 
+    peak, peak_src = measured_peak()
+
+    # ---- the W8A8 linear layer (INT8 GEMM with 128x128 block scales) on a Wan2.1-14B
+    # feed-forward shape: the quantiser + GEMM call, and the GEMM kernel alone
+    w8a8 = None
+    if args.linear_workload != "none":
+        del dq, dk, dv
+        lw = LINEAR_WORKLOADS[args.linear_workload]
+        x_bits, w_bits = make_linear_workload(lw)
+        dx = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        dw = torch.from_numpy(w_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        del x_bits, w_bits
+        wq = sa.sa_w8a8_quantize(dw)
+        xq = sa.sa_w8a8_quantize(dx)
+        dy = torch.empty((lw.M, lw.N), dtype=torch.bfloat16, device=dev)
+
+        def timed(fn):
+            for _ in range(args.warmup):
+                fn()
+            barrier()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            t1.record(stream)
+            barrier()
+            return slowest(t0.elapsed_time(t1) / 1e3 / args.steps)
+
+        t_lin = timed(lambda: sa.sa_w8a8_linear(dx, wq, out=dy))
+        t_gemm = timed(lambda: sa.sa_w8a8_gemm(xq, wq, lw.K, out=dy))
+        assert sa.sa_get_device_status() == 0
+        gemm_tops = lw.ops / t_gemm / 1e12
+        w8a8 = {"workload": lw.name, "M": lw.M, "N": lw.N, "K": lw.K, "ops": lw.ops,
+                "step": "sa_w8a8_linear: x block quantisation + block-scaled INT8 GEMM, bf16 out",
+                "value": whole_job_tops(lw.ops, world, t_lin), "unit": "TOPS", "ms": t_lin * 1e3,
+                "roofline": {"bound": "tensor", "kernel": "w8a8_gemm_kernel", "achieved": gemm_tops,
+                             "peak": peak, "unit": "TOPS", "frac": gemm_tops / peak, "peak_source": peak_src,
+                             "ms_per_launch": t_gemm * 1e3}}
+        del dx, dw, xq, wq, dy
+
     ops_rank = w.dense_ops
     value = whole_job_tops(ops_rank, world, t_step)
-    peak, peak_src = measured_peak()
     achieved = ops_rank / t_attn / 1e12
     kernel = "attn_fwd_kernel" if w.mask_density is not None else "attn_pairs_kernel"
     traffic = recorded_traffic(kernel, w.name)
@@ -376,6 +419,8 @@ def main():
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
         }
+        if w8a8 is not None:
+            line["w8a8"] = w8a8
         if w.mask_density is not None and m is not None:
             kept = int(m.sum())
             exe = 4.0 * w.d * 128 * 64 * kept

@@ -347,38 +347,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             float acc[128];
 #pragma unroll
             for (int c = 0; c < 128; ++c) acc[c] = 0.0f;
+            // the block scales of k-block b + 1 load while k-block b is processed
+            const float *sxr = sx + int64_t(live ? mb : 0) * nkb, *swr = sw + int64_t(live ? nb : 0) * nkb;
+            float sx_next = live ? sxr[0] : 0.0f, sw_next = live ? swr[0] : 0.0f;
             for (int b = 0; b < nkb; ++b, ++g) {
                 const uint32_t ab = g & 1;
-                const float s = live ? sx[int64_t(mb) * nkb + b] * sw[int64_t(nb) * nkb + b] : 0.0f;
+                const float s = sx_next * sw_next;  // the block's scale product, as in the definition
+                if (live && b + 1 < nkb) {
+                    sx_next = sxr[b + 1];
+                    sw_next = swr[b + 1];
+                }
                 if (ok) ok = mbar_wait(bar(kBarAccFull + ab), (g >> 1) & 1, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
-                if (ok) tc_fence_after();
+                const uint32_t acc_empty = cluster_addr(bar(kBarAccEmpty + ab), 0);
+                if (!ok) {
+                    if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty);
+                    continue;
+                }
+                tc_fence_after();
                 const uint32_t ta = tmem + lane_addr + ab * kTileN + half * 128;
                 // 16-column chunks: chunk q + 1 is loading while chunk q is folded in
                 uint32_t va[16], vb[16];
-                if (ok) tmem_ld16_nowait(ta, va);
+                tmem_ld16_nowait(ta, va);
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint32_t(&cur)[16] = (q & 1) ? vb : va;
                     uint32_t(&nxt)[16] = (q & 1) ? va : vb;
-                    if (ok) {
-                        tmem_wait_ld();
-                        regs_ready16(cur);
-                    }
+                    tmem_wait_ld();
+                    regs_ready16(cur);
                     if (q == 7) {
                         // the warp's whole block is in registers: release the accumulator
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive_cluster_relaxed(cluster_addr(bar(kBarAccEmpty + ab), 0));
-                    } else if (ok) {
+                        if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty);
+                    } else {
                         tmem_ld16_nowait(ta + 16 * (q + 1), nxt);
                     }
-                    if (ok) {
 #pragma unroll
-                        for (int i = 0; i < 16; i += 2)
-                            fma2(acc[16 * q + i], acc[16 * q + i + 1], __int2float_rn(int(cur[i])),
-                                 __int2float_rn(int(cur[i + 1])), s, s, acc[16 * q + i], acc[16 * q + i + 1]);
-                    }
+                    for (int i = 0; i < 16; i += 2)
+                        fma2(acc[16 * q + i], acc[16 * q + i + 1], __int2float_rn(int(cur[i])),
+                             __int2float_rn(int(cur[i + 1])), s, s, acc[16 * q + i], acc[16 * q + i + 1]);
                 }
             }
             // bf16 row of 128 columns: 16-byte stores, columns < N

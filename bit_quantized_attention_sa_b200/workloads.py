@@ -161,6 +161,10 @@ LINEAR_WORKLOADS = {
     "small-m300-n264-k1000": LinearWorkload("small-m300-n264-k1000", 300, 264, 1000, seed=2000),
     "wan14b-720p-ffn-up-m75600-n13824-k5120": LinearWorkload(
         "wan14b-720p-ffn-up-m75600-n13824-k5120", 75600, 13824, 5120, seed=2001),
+    # a 16384-token slice of the same layer (codes of x and w together exceed L2), for
+    # profiler captures that must stay small
+    "wan14b-ffn-up-m16384-n13824-k5120": LinearWorkload(
+        "wan14b-ffn-up-m16384-n13824-k5120", 16384, 13824, 5120, seed=2002),
 }
 
 
