@@ -68,6 +68,8 @@ def _load():
         lib.sa_oracle_w8a8_quantize.argtypes = [P, I64, I64, P, P]
         lib.sa_oracle_w8a8_quantize.restype = None
         lib.sa_oracle_w8a8_gemm_rows.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+        lib.sa_oracle_sla_linear_rows.argtypes = [P, P, P, I, I, I, I, P, I, P, P, I64, P]
+        lib.sa_oracle_sla_linear_rows.restype = None
         lib.sa_oracle_w8a8_gemm_rows.restype = None
         _lib = lib
     return _lib
@@ -229,3 +231,20 @@ def w8a8_gemm_rows(xq, wq, K: int, rows) -> np.ndarray:
     _load().sa_oracle_w8a8_gemm_rows(_ptr(x8), _ptr(sx), _ptr(w8), _ptr(sw), M, N, K, _ptr(rows),
                                      rows.size, _ptr(y))
     return y
+
+
+def sla_linear_rows(q, k, v, classes: np.ndarray, phi: int, proj: np.ndarray | None, rows) -> np.ndarray:
+    """SLA linear branch for rows [(bh, r), ...]: kernelised linear attention over the
+    marginal blocks (classes == 1) with feature map phi (0 softmax, 1 elu+1), projected by
+    proj (fp32 [d, d], None = identity).  Returns fp64 [len(rows), d]."""
+    B, H, N, d = q.shape
+    rows = _rows_array(rows, B, H, N)
+    classes = np.ascontiguousarray(classes, dtype=np.uint8)
+    assert classes.shape == (B, H, -(-N // QBLK), -(-N // KBLK))
+    if proj is not None:
+        proj = np.ascontiguousarray(proj, dtype=np.float32)
+        assert proj.shape == (d, d)
+    out = np.zeros((rows.shape[0], d), np.float64)
+    _load().sa_oracle_sla_linear_rows(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, _ptr(classes), int(phi),
+                                      _ptr(proj), _ptr(rows), rows.shape[0], _ptr(out))
+    return out

@@ -44,7 +44,10 @@
  * stable sort (ties included), invariants (scaling Q, swapping key blocks) and a planted
  * key block (tests/test_oracle_mask.py).  W8A8 linear layer (end of file): quantiser
  * against a numpy restatement, exact-integer and single-k-block closed forms, zero blocks,
- * error against the fp64 product (tests/test_oracle_w8a8.py).
+ * error against the fp64 product (tests/test_oracle_w8a8.py).  SLA linear branch (end of
+ * file): the factorised form in numpy, closed forms (one key, identical keys, no marginal
+ * block), invariants (constant V columns, W = identity vs W applied afterwards) and the
+ * class semantics (tests/test_oracle_sla.py).
  */
 #include <fenv.h>
 #include <math.h>
@@ -571,4 +574,95 @@ void sa_oracle_w8a8_gemm_rows(const int8_t *x8, const float *sx, const int8_t *w
             y[ri * N + n] = acc;
         }
     }
+}
+
+/* ------------------------------------------------------------------------------------
+ * SLA linear-attention branch (the "marginal" blocks of Sparse-Linear Attention).
+ *
+ * Sources: NetEase article on the TurboDiffusion release, attention-acceleration section:
+ * SLA combines sparse attention with linear attention, and its figure caption splits the
+ * attention weights into three classes computed at different costs; "AIGC weekend
+ * special 5.10" section 1.2 Method item (2): SLA is a trainable sparse *linear* attention
+ * used on top of SageAttention.  The pages give no formula for the linear part.
+ *
+ * Reading: the classes come per (128-query block i, 64-key block j) in a uint8 map:
+ * 0 = negligible (skipped), 1 = marginal (linear attention), >= 2 = critical (the sparse
+ * quantised attention above).  The marginal part is kernelised linear attention with a
+ * feature map phi applied to each row's d features:
+ *     w_t = phi(q_r) . phi(k_t) over the keys t < N of the row's marginal blocks,
+ *     O_lin[r] = sum_t w_t v_t / sum_t w_t          (0 when the row has no marginal key),
+ * and the branch's output is O_lin projected by a d x d matrix W (a trained layer in
+ * SLA; here any given matrix, the identity when NULL): out[r][c] = sum_e W[c][e] O_lin[r][e].
+ * phi = 0: softmax over the features, phi(x)_a = exp(x_a - max x) / sum_b exp(x_b - max x);
+ * phi = 1: elu(x) + 1, i.e. x + 1 for x > 0 and exp(x) otherwise.  Both are positive, so
+ * sum_t w_t > 0 whenever the row has a marginal key.
+ * This is the weighted-average form written out in fp64 per row; it equals the
+ * factorised form phi(q)^T (sum_t phi(k_t) v_t^T) / (phi(q) . sum_t phi(k_t)) by
+ * associativity, which is how a fast implementation evaluates it.
+ * ------------------------------------------------------------------------------------ */
+
+static void phi_row(const uint16_t *x, int d, int phi, double *out)
+{
+    if (phi == 0) {
+        double mx = -INFINITY;
+        for (int a = 0; a < d; ++a) {
+            const double v = (double)bf16_to_f32(x[a]);
+            if (v > mx) mx = v;
+        }
+        double sum = 0.0;
+        for (int a = 0; a < d; ++a) {
+            out[a] = exp((double)bf16_to_f32(x[a]) - mx);
+            sum += out[a];
+        }
+        for (int a = 0; a < d; ++a) out[a] /= sum;
+    } else {
+        for (int a = 0; a < d; ++a) {
+            const double v = (double)bf16_to_f32(x[a]);
+            out[a] = v > 0.0 ? v + 1.0 : exp(v);
+        }
+    }
+}
+
+/* classes: uint8 [B,H,nq,nk]; proj: fp32 [d][d] (row = output feature) or NULL;
+ * rows: (bh, r) pairs; out: fp64 [nrows, d]. */
+void sa_oracle_sla_linear_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int H,
+                               int N, int d, const uint8_t *classes, int phi, const float *proj,
+                               const int64_t *rows, int64_t nrows, double *out)
+{
+    (void)B; (void)H;
+    const int64_t nq = cdiv64(N, QBLK), nk = cdiv64(N, KBLK);
+    double *pq = (double *)malloc(sizeof(double) * (size_t)d);
+    double *pk = (double *)malloc(sizeof(double) * (size_t)d);
+    double *ol = (double *)malloc(sizeof(double) * (size_t)d);
+    for (int64_t n = 0; n < nrows; ++n) {
+        const int64_t bh = rows[2 * n], r = rows[2 * n + 1];
+        const int64_t i = r / QBLK;
+        const uint8_t *crow = classes + (bh * nq + i) * nk;
+        phi_row(q + (bh * N + r) * d, d, phi, pq);
+        double den = 0.0;
+        for (int c = 0; c < d; ++c) ol[c] = 0.0;
+        for (int64_t t = 0; t < N; ++t) {
+            if (crow[t / KBLK] != 1) continue;
+            phi_row(k + (bh * N + t) * d, d, phi, pk);
+            double w = 0.0;
+            for (int a = 0; a < d; ++a) w += pq[a] * pk[a];
+            den += w;
+            const uint16_t *vt = v + (bh * N + t) * d;
+            for (int c = 0; c < d; ++c) ol[c] += w * (double)bf16_to_f32(vt[c]);
+        }
+        double *o = out + n * d;
+        for (int c = 0; c < d; ++c) ol[c] = den > 0.0 ? ol[c] / den : 0.0;
+        for (int c = 0; c < d; ++c) {
+            if (!proj) {
+                o[c] = ol[c];
+                continue;
+            }
+            double acc = 0.0;
+            for (int e = 0; e < d; ++e) acc += (double)proj[c * d + e] * ol[e];
+            o[c] = acc;
+        }
+    }
+    free(pq);
+    free(pk);
+    free(ol);
 }
