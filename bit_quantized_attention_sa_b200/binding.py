@@ -37,6 +37,8 @@ _lib.sa_debug_pool.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_w8a8_quantize.argtypes = [_P, _I, _I, _P, _P, _P]
 _lib.sa_w8a8_gemm.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P, _P]
 _lib.sa_w8a8_linear.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
+_lib.sa_sla_linear.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]
+_lib.sa_sla_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P]
 _lib.sa_debug_wait_timeout.argtypes = [_I, _P]
 _lib.sa_debug_exp2_poly.argtypes = [_P, _P, _I, _P]
 _lib.sa_get_device_status.argtypes = []
@@ -49,7 +51,7 @@ _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
               "sa_attn_fwd_quantized",
-              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
+              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_sla_linear", "sa_sla_fwd", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
 
@@ -303,6 +305,48 @@ def sa_w8a8_linear(x: torch.Tensor, wq, out=None):
     _check(_lib.sa_w8a8_linear(_ptr(x), _ptr(wc), _ptr(ws), M, N, K, _ptr(y), _stream(x.device)),
            "sa_w8a8_linear")
     return y
+
+
+SA_PHI_SOFTMAX, SA_PHI_ELU1 = 0, 1
+
+
+def _sla_args(q, k, v, classes, proj):
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, name)
+    B, H, N, d = _dims(q)
+    if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
+        raise ValueError("q, k and v shapes differ")
+    _need(classes, torch.uint8, "classes")
+    if tuple(classes.shape) != (B, H, -(-N // 128), -(-N // 64)):
+        raise ValueError("classes must be uint8 [B, H, ceil(N/128), ceil(N/64)]")
+    if proj is not None:
+        _need(proj, torch.float32, "proj")
+        if tuple(proj.shape) != (d, d):
+            raise ValueError("proj must be fp32 [d, d]")
+    return B, H, N, d
+
+
+def sa_sla_linear(q, k, v, classes, phi: int = SA_PHI_SOFTMAX, proj=None, out=None):
+    """SLA linear branch: fp32 [B,H,N,d] = proj-projected linear attention of each row over
+    its marginal blocks (classes == 1); phi SA_PHI_SOFTMAX or SA_PHI_ELU1."""
+    B, H, N, d = _sla_args(q, k, v, classes, proj)
+    o = torch.empty((B, H, N, d), dtype=torch.float32, device=q.device) if out is None else out
+    _need(o, torch.float32, "out")
+    _check(_lib.sa_sla_linear(_ptr(q), _ptr(k), _ptr(v), _ptr(classes), B, H, N, d, int(phi), _ptr(proj), _ptr(o),
+                              _stream(q.device)), "sa_sla_linear")
+    return o
+
+
+def sa_sla_fwd(q, k, v, classes, sm_scale: float | None = None, phi: int = SA_PHI_SOFTMAX, proj=None, out=None):
+    """SLA forward: bf16 [B,H,N,d] = sparse quantised attention over the critical blocks
+    (classes >= 2) + the projected linear branch over the marginal blocks (classes == 1)."""
+    B, H, N, d = _sla_args(q, k, v, classes, proj)
+    scale = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    _need(o, torch.bfloat16, "out")
+    _check(_lib.sa_sla_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, scale, _ptr(classes), int(phi),
+                           _ptr(proj), _stream(q.device)), "sa_sla_fwd")
+    return o
 
 
 def sa_debug_qk_s32(q_i8, k_i8, N: int):

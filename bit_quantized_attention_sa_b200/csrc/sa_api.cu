@@ -516,6 +516,59 @@ sa_status sa_w8a8_linear(const void *x, const int8_t *w_codes, const float *w_sc
     return w8a8_gemm_checked(xc, xs, w_codes, w_scales, M, N, K, y, st);
 }
 
+static sa_status check_sla(const Shape &s, int phi, std::initializer_list<const void *> ptrs)
+{
+    if (phi != 0 && phi != 1) return SA_ERR_INVALID_ARG;
+    if (s.nk() > kMaskMaxKeyBlocks) return SA_ERR_UNSUPPORTED;
+    return check_ptrs(ptrs);
+}
+
+sa_status sa_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, int B, int H, int N,
+                        int d, int phi, const float *proj, float *out, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (!classes) return SA_ERR_INVALID_ARG;
+    if ((r = check_sla(s, phi, {q, k, v, out})) != SA_OK) return r;
+    if (proj && (r = check_ptrs({proj})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    const size_t sb = align256(sla_state_bytes(s));
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(sb + sla_sum_bytes(s), &ws)) != SA_OK) return r;
+    return launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws),
+                             reinterpret_cast<float *>(ws + sb), false, out,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
+sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B, int H, int N, int d,
+                     float sm_scale, const uint8_t *classes, int phi, const float *proj, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale) || !classes) return SA_ERR_INVALID_ARG;
+    if ((r = check_sla(s, phi, {q, k, v, o})) != SA_OK) return r;
+    if (proj && (r = check_ptrs({proj})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    // workspace: [attention prologue | keep mask | states | summed states]
+    const size_t attn = align256(ws_layout(s).total);
+    const size_t nmask = size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk());
+    const size_t mb = align256(nmask), sb = align256(sla_state_bytes(s));
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(attn + mb + sb + sla_sum_bytes(s), &ws)) != SA_OK) return r;
+    uint8_t *keep = ws + attn;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_sla_critical(classes, int64_t(nmask), keep, st) != cudaSuccess) return SA_ERR_CUDA;
+    if ((r = attn_fwd_device(q, k, v, o, s, sm_scale, keep, st)) != SA_OK) return r;
+    return launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws + attn + mb),
+                             reinterpret_cast<float *>(ws + attn + mb + sb), true, o, st) == cudaSuccess
+               ? SA_OK
+               : SA_ERR_CUDA;
+}
+
 sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
                           int32_t *s_out, void *stream)
 {

@@ -68,6 +68,16 @@ constexpr int kW8a8BoxRows = 128;
 cudaError_t launch_w8a8_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, const float *sx,
                              const float *sw, int M, int N, int nkb, void *y, cudaStream_t st);
 cudaError_t read_and_clear_w8a8_status(int *status);
+// ---- SLA linear branch (sa_sla.cu)
+size_t sla_state_bytes(const Shape &s);  // per-key-block states, fp32
+size_t sla_sum_bytes(const Shape &s);    // per-query-block summed states, fp32
+// The branch for all rows: fp32 out [B,H,N,d] (add_into_bf16 false) or added to the bf16
+// out (true).  classes uint8 [B,H,nq,nk] (1 = marginal); proj fp32 [d][d] or null.
+cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, const Shape &s,
+                              int phi, const float *proj, float *state, float *sums, bool add_into_bf16, void *out,
+                              cudaStream_t st);
+// keep[e] = classes[e] >= 2 (the sparse part's block mask), n entries.
+cudaError_t launch_sla_critical(const uint8_t *classes, int64_t n, uint8_t *keep, cudaStream_t st);
 // Reads and clears the device status word of the current device (synchronous).
 cudaError_t read_and_clear_status(int *status);
 

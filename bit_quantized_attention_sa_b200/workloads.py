@@ -192,3 +192,20 @@ def make_linear_inputs(M: int, N: int, K: int, seed: int = 0, outliers: bool = T
 
 def make_linear_workload(w: LinearWorkload):
     return make_linear_inputs(w.M, w.N, w.K, seed=w.seed)
+
+
+def make_sla_classes(B: int, H: int, N: int, p_critical: float, p_marginal: float, seed: int = 0):
+    """uint8 [B,H,nq,nk] SLA block classes: each (128-query x 64-key) block is critical (2)
+    with probability p_critical, marginal (1) with probability p_marginal, else negligible
+    (0), from one ``Generator(PCG64(seed))`` draw of uniforms; the diagonal blocks
+    j in {2i, 2i+1} are always critical."""
+    nq, nk = -(-N // QBLK), -(-N // KBLK)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    u = rng.random((B, H, nq, nk), dtype=np.float32)
+    cls = np.where(u < np.float32(p_critical), 2, np.where(u < np.float32(p_critical + p_marginal), 1, 0))
+    cls = cls.astype(np.uint8)
+    for i in range(nq):
+        for j in (2 * i, 2 * i + 1):
+            if j < nk:
+                cls[:, :, i, j] = 2
+    return cls

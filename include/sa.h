@@ -182,6 +182,35 @@ sa_status sa_w8a8_gemm(const int8_t *x_codes, const float *x_scales, const int8_
 sa_status sa_w8a8_linear(const void *x, const int8_t *w_codes, const float *w_scales, int M, int N,
                          int K, void *y, void *stream);
 
+/* ---- SLA: sparse quantised attention on the critical blocks plus linear attention on the
+ * marginal blocks.
+ * Sources: NetEase article on the TurboDiffusion release, attention-acceleration section
+ * (SLA combines sparse and linear attention; its figure caption splits the attention
+ * weights into three classes handled at different costs); "AIGC weekend special 5.10"
+ * section 1.2 Method item (2) (SLA runs on top of SageAttention).  The pages give no
+ * formula for the linear part.  Reading: block classes come per (128-query block,
+ * 64-key block) in classes uint8 [B,H,nq,nk] (device): 0 = negligible (skipped), 1 =
+ * marginal (linear attention), >= 2 = critical (sparse quantised attention).  The linear
+ * part is kernelised linear attention over the keys of the row's marginal blocks,
+ *     O_lin[r] = sum_t w_t v_t / sum_t w_t,  w_t = phi(q_r) . phi(k_t)   (0 if no such key),
+ * with phi = SA_PHI_SOFTMAX (softmax over the d features of a row) or SA_PHI_ELU1
+ * (elu(x) + 1), projected by W: out[r][c] = sum_e W[c][e] O_lin[r][e], W fp32 [d][d]
+ * (device; NULL = identity; in SLA a trained layer).  Evaluated in fp32 in the factorised
+ * form phi(q)^T (sum_t phi(k_t) v_t^T) / (phi(q) . sum_t phi(k_t)).
+ * Needs ceil(N/64) <= 4096 (else SA_ERR_UNSUPPORTED).  Uses the library workspace:
+ * 69,632 bytes per 64-key block and per 128-query block of every head. */
+enum { SA_PHI_SOFTMAX = 0, SA_PHI_ELU1 = 1 };
+
+/* The linear branch alone: out fp32 [B,H,N,d] (device, caller-owned) = W O_lin. */
+sa_status sa_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, int B, int H,
+                        int N, int d, int phi, const float *proj, float *out, void *stream);
+
+/* The SLA forward: o bf16 [B,H,N,d] = the quantised attention of sa_attn_fwd restricted to
+ * the critical blocks (a row without one gives 0), plus the projected linear branch,
+ * added in fp32 and rounded once to bf16. */
+sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B, int H, int N, int d,
+                     float sm_scale, const uint8_t *classes, int phi, const float *proj, void *stream);
+
 /* Debug: the int32 S = q_i8 . k_i8^T tiles computed by the same tcgen05 INT8 path the
  * attention kernel uses, stored to s_out int32 [B,H,Npad,Npad] (padded rows/keys
  * included).  For bit-exact checks on small problems only.  Allocates nothing. */

@@ -85,3 +85,17 @@ def test_w8a8_argument_errors(libsa):
     assert lib.sa_w8a8_linear(FAKE, FAKE, FAKE, 128, 12, 128, FAKE, None) == 2
     assert lib.sa_w8a8_linear(FAKE, FAKE, FAKE, 128, 128, 100, FAKE, None) == 2
     assert lib.sa_w8a8_linear(ODD, FAKE, FAKE, 128, 128, 128, FAKE, None) == 3
+
+
+def test_sla_argument_errors(libsa):
+    lib = libsa.raw_library()
+    f = ctypes.c_float(0.088)
+    # phi must be 0 or 1; classes required; at most 4096 key blocks; d = 128; aligned
+    assert lib.sa_sla_linear(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 2, None, FAKE, None) == 1
+    assert lib.sa_sla_linear(FAKE, FAKE, FAKE, None, 1, 1, 128, 128, 0, None, FAKE, None) == 1
+    assert lib.sa_sla_linear(FAKE, FAKE, FAKE, FAKE, 1, 1, 4096 * 64 + 1, 128, 0, None, FAKE, None) == 2
+    assert lib.sa_sla_linear(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, None, FAKE, None) == 2
+    assert lib.sa_sla_linear(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0, ODD, FAKE, None) == 3
+    assert lib.sa_sla_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, ctypes.c_float(0.0), FAKE, 0, None, None) == 1
+    assert lib.sa_sla_fwd(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, f, FAKE, 1, None, None) == 3
+    assert lib.sa_sla_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, f, FAKE, 1, None, None) == 1
