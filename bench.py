@@ -28,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from bit_quantized_attention_sa_b200.workloads import (LINEAR_WORKLOADS, WORKLOADS, make_linear_workload,  # noqa: E402
-                                                       make_workload)
+                                                       make_sla_classes, make_workload)
 
 METRIC = "quantized attention TOPS (4·H·N²·d/s) and % of B200 dense INT8/FP8 peak"
 DEFAULT_WORKLOAD = "wan14b-720p-h40-n75600"
@@ -224,6 +224,7 @@ def main():
     ap.add_argument("--oracle-rows", type=int, default=64,
                     help="query rows in the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sla", action="store_true", help="skip the SLA forward timing")
     ap.add_argument("--linear-workload", default=DEFAULT_LINEAR, choices=list(LINEAR_WORKLOADS) + ["none"],
                     help="W8A8 linear layer timed beside the attention step ('none' skips it)")
     args = ap.parse_args()
@@ -345,6 +346,40 @@ def main():
 
     peak, peak_src = measured_peak()
 
+    # ---- the SLA forward on the same inputs: sparse quantised attention over the critical
+    # blocks plus linear attention over the marginal blocks, projected
+    sla = None
+    if not args.no_sla:
+        p_crit, p_marg = 0.0965, 0.4
+        cls = torch.from_numpy(make_sla_classes(w.B, w.H, w.N, p_crit, p_marg, seed=w.seed + 1)).to(dev)
+        proj = torch.from_numpy((np.random.default_rng(w.seed).standard_normal((w.d, w.d)) / math.sqrt(w.d))
+                                .astype(np.float32)).to(dev)
+        lin_out = torch.empty(shape, dtype=torch.float32, device=dev)
+
+        def timed_sla(fn):
+            for _ in range(args.warmup):
+                fn()
+            barrier()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            t1.record(stream)
+            barrier()
+            return slowest(t0.elapsed_time(t1) / 1e3 / args.steps)
+
+        t_sla = timed_sla(lambda: sa.sa_sla_fwd(dq, dk, dv, cls, w.sm_scale, proj=proj, out=do))
+        t_lin = timed_sla(lambda: sa.sa_sla_linear(dq, dk, dv, cls, proj=proj, out=lin_out))
+        assert sa.sa_get_device_status() == 0
+        sla = {"step": "sa_sla_fwd: quantised attention on critical blocks + projected linear attention on "
+                       "marginal blocks (phi = softmax over features)",
+               "classes": {"critical": float((cls >= 2).float().mean().item()),
+                           "marginal": float((cls == 1).float().mean().item()),
+                           "recipe": f"critical p={p_crit} (+ diagonal), marginal p={p_marg}, else skipped"},
+               "ms": t_sla * 1e3, "linear_branch_ms": t_lin * 1e3,
+               "dense_equivalent_tops": whole_job_tops(w.dense_ops, world, t_sla)}
+        del cls, proj, lin_out
+
     # ---- the W8A8 linear layer (INT8 GEMM with 128x128 block scales) on a Wan2.1-14B
     # feed-forward shape: the quantiser + GEMM call, and the GEMM kernel alone
     w8a8 = None
@@ -419,6 +454,8 @@ def main():
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
         }
+        if sla is not None:
+            line["sla"] = sla
         if w8a8 is not None:
             line["w8a8"] = w8a8
         if w.mask_density is not None and m is not None:

@@ -133,37 +133,50 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// grid (kSumChunks, ceil(nq / 16), BH), 256 threads; dynamic shared memory nk uint16.
+// grid (kSumChunks, ceil(nq / 16), BH), 256 threads; dynamic shared memory nk uint32.
 // A_i (chunk) = sum over j ascending of the states of the blocks with classes[i][j] == 1.
 __global__ void __launch_bounds__(256)
     sla_state_sum_kernel(const float *__restrict__ state, const uint8_t *__restrict__ classes, int nq, int nk,
                          float *__restrict__ sums)
 {
-    extern __shared__ uint16_t marg_bits[];  // bit g: query block i0 + g has class 1 at j
+    extern __shared__ uint32_t marg_bits[];  // bit g: query block i0 + g has class 1 at j
     const int64_t bh = blockIdx.z;
     const int cc = blockIdx.x, i0 = blockIdx.y * kSumGroup, tid = threadIdx.x;
     const int ng = min(kSumGroup, nq - i0);
     for (int j = tid; j < nk; j += blockDim.x) {
         uint32_t bits = 0;
         for (int g = 0; g < ng; ++g) bits |= uint32_t(classes[(bh * nq + i0 + g) * int64_t(nk) + j] == 1) << g;
-        marg_bits[j] = uint16_t(bits);
+        marg_bits[j] = bits;
     }
     __syncthreads();
     float4 acc[kSumGroup];
 #pragma unroll
     for (int g = 0; g < kSumGroup; ++g) acc[g] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     const float *src = state + bh * int64_t(nk) * kStateFloats + cc * kSumChunk + 4 * tid;
-    for (int j = 0; j < nk; ++j) {
-        const uint32_t bits = marg_bits[j];
-        if (bits == 0) continue;
-        const float4 h = __ldg(reinterpret_cast<const float4 *>(src + int64_t(j) * kStateFloats));
+    // 8 key blocks per step: their loads are all in flight before the first is added
+    constexpr int kAhead = 8;
+    for (int j0 = 0; j0 < nk; j0 += kAhead) {
+        uint32_t bits[kAhead];
+        float4 h[kAhead];
 #pragma unroll
-        for (int g = 0; g < kSumGroup; ++g) {
-            if ((bits >> g) & 1u) {
-                acc[g].x += h.x;
-                acc[g].y += h.y;
-                acc[g].z += h.z;
-                acc[g].w += h.w;
+        for (int u = 0; u < kAhead; ++u) {
+            bits[u] = j0 + u < nk ? marg_bits[j0 + u] : 0u;
+            h[u] = bits[u] ? __ldg(reinterpret_cast<const float4 *>(src + int64_t(j0 + u) * kStateFloats))
+                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+        // keeps the compiler from sinking each load to its first use
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) asm volatile("" ::"f"(h[u].x), "f"(h[u].y), "f"(h[u].z), "f"(h[u].w));
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+#pragma unroll
+            for (int g = 0; g < kSumGroup; ++g) {
+                if ((bits[u] >> g) & 1u) {
+                    acc[g].x += h[u].x;
+                    acc[g].y += h[u].y;
+                    acc[g].z += h[u].z;
+                    acc[g].w += h[u].w;
+                }
             }
         }
     }
@@ -329,7 +342,7 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
         if ((e = cudaFuncSetAttribute(sla_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(state_smem))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_state_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(sizeof(uint16_t) * kMaskMaxKeyBlocks))) != cudaSuccess ||
+                                      int(sizeof(uint32_t) * kMaskMaxKeyBlocks))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_apply_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(kApplySmemBytes))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_apply_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -343,7 +356,7 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
         static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), N, nk, phi, state);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     sla_state_sum_kernel<<<dim3(unsigned(kSumChunks), unsigned((nq + kSumGroup - 1) / kSumGroup), unsigned(s.BH())),
-                           256, sizeof(uint16_t) * size_t(nk), st>>>(state, classes, nq, nk, sums);
+                           256, sizeof(uint32_t) * size_t(nk), st>>>(state, classes, nq, nk, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 ga(unsigned(nq), unsigned(s.BH()));
     if (add_into_bf16)
