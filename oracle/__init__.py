@@ -68,6 +68,10 @@ def _load():
         lib.sa_oracle_w8a8_quantize.argtypes = [P, I64, I64, P, P]
         lib.sa_oracle_w8a8_quantize.restype = None
         lib.sa_oracle_w8a8_gemm_rows.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
+        lib.sa_oracle_attn_rows_causal.argtypes = lib.sa_oracle_attn_rows.argtypes
+        lib.sa_oracle_attn_rows_causal.restype = None
+        lib.sa_oracle_exact_rows_causal.argtypes = lib.sa_oracle_exact_rows.argtypes
+        lib.sa_oracle_exact_rows_causal.restype = None
         lib.sa_oracle_sla_linear_rows.argtypes = [P, P, P, I, I, I, I, P, I, P, P, I64, P]
         lib.sa_oracle_sla_linear_rows.restype = None
         lib.sa_oracle_w8a8_gemm_rows.restype = None
@@ -130,9 +134,9 @@ def _rows_array(rows, B, H, N):
 
 
 def attn_rows(qk, vq, N: int, sm_scale: float, rows, mask: np.ndarray | None = None,
-              group: int = 2) -> np.ndarray:
-    """Quantised attention for rows [(bh, r), ...] from quantize_qk / quantize_v outputs.
-    Returns fp32 [len(rows), d]."""
+              group: int = 2, causal: bool = False) -> np.ndarray:
+    """Quantised attention for rows [(bh, r), ...] from quantize_qk / quantize_v outputs
+    (causal: row r takes the keys t <= r only).  Returns fp32 [len(rows), d]."""
     q_i8, q_scale, k_i8, k_scale = qk[0], qk[1], qk[2], qk[3]
     v_t, v_scale = vq
     B, H, _, d = q_i8.shape
@@ -141,20 +145,24 @@ def attn_rows(qk, vq, N: int, sm_scale: float, rows, mask: np.ndarray | None = N
         mask = np.ascontiguousarray(mask, dtype=np.uint8)
         assert mask.shape == (B, H, -(-N // QBLK), -(-N // KBLK))
     out = np.zeros((rows.shape[0], d), np.float32)
-    _load().sa_oracle_attn_rows(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale),
+    fn = _load().sa_oracle_attn_rows_causal if causal else _load().sa_oracle_attn_rows
+    fn(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale),
                                 _ptr(v_t), _ptr(v_scale), B, H, N, d, float(sm_scale),
                                 _ptr(mask), int(group), _ptr(rows), rows.shape[0], _ptr(out))
     return out
 
 
-def exact_rows(q, k, v, sm_scale: float, rows, mask: np.ndarray | None = None) -> np.ndarray:
-    """fp64 softmax(q K^T sm_scale) V from the bf16 inputs for rows [(bh, r), ...]."""
+def exact_rows(q, k, v, sm_scale: float, rows, mask: np.ndarray | None = None,
+               causal: bool = False) -> np.ndarray:
+    """fp64 softmax(q K^T sm_scale) V from the bf16 inputs for rows [(bh, r), ...]
+    (causal: row r over the keys t <= r)."""
     B, H, N, d = q.shape
     rows = _rows_array(rows, B, H, N)
     if mask is not None:
         mask = np.ascontiguousarray(mask, dtype=np.uint8)
     out = np.zeros((rows.shape[0], d), np.float64)
-    _load().sa_oracle_exact_rows(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(sm_scale),
+    fn = _load().sa_oracle_exact_rows_causal if causal else _load().sa_oracle_exact_rows
+    fn(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, float(sm_scale),
                                  _ptr(mask), _ptr(rows), rows.shape[0], _ptr(out))
     return out
 

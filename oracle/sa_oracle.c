@@ -277,10 +277,10 @@ static int64_t kept_blocks(const uint8_t *mask, int64_t bh, int64_t i, int64_t n
  * column is reproduced and the normalised weights sum to one up to fp32 rounding.
  * reading: alpha is applied whenever the running max grows (no lazy rescaling, which
  * would push 448*P past the e4m3 range). */
-void sa_oracle_attn_rows(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
-                         const float *k_scale, const uint8_t *v_fp8_t, const float *v_scale,
-                         int B, int H, int N, int d, float sm_scale, const uint8_t *mask,
-                         int group, const int64_t *rows, int64_t nrows, float *out)
+static void attn_rows_impl(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                           const float *k_scale, const uint8_t *v_fp8_t, const float *v_scale,
+                           int B, int H, int N, int d, float sm_scale, const uint8_t *mask,
+                           int group, int causal, const int64_t *rows, int64_t nrows, float *out)
 {
     fesetround(FE_TONEAREST);
     (void)B; (void)H;
@@ -300,7 +300,15 @@ void sa_oracle_attn_rows(const int8_t *q_i8, const float *q_scale, const int8_t 
         const int8_t *kh = k_i8 + bh * Npad * d;
         const uint8_t *vt = v_fp8_t + bh * d * Npad;
         const float sq = q_scale[bh * nq + i];
-        const int64_t nkept = kept_blocks(mask, bh, i, nq, nk, blocks);
+        int64_t nkept = kept_blocks(mask, bh, i, nq, nk, blocks);
+        if (causal) {
+            /* reading: causal rows keep the blocks up to their tile's diagonal pair,
+             * j <= 2i + 1, so the steps are the same pairs as without causality */
+            int64_t n2 = 0;
+            for (int64_t g = 0; g < nkept; ++g)
+                if (blocks[g] <= 2 * i + 1) blocks[n2++] = blocks[g];
+            nkept = n2;
+        }
 
         float m = -INFINITY, l = 0.0f;
         for (int c = 0; c < d; ++c) acc[c] = 0.0f;
@@ -312,7 +320,7 @@ void sa_oracle_attn_rows(const int8_t *q_i8, const float *q_scale, const int8_t 
             for (int64_t g = g0; g < g1; ++g) {
                 const int64_t j = blocks[g];
                 const float sk = k_scale[bh * nk + j];
-                for (int64_t t = j * KBLK; t < (j + 1) * KBLK && t < N; ++t) {
+                for (int64_t t = j * KBLK; t < (j + 1) * KBLK && t < N && (!causal || t <= r); ++t) {
                     int32_t S = 0;
                     for (int c = 0; c < d; ++c) S += (int32_t)qrow[c] * (int32_t)kh[t * d + c];
                     float sc = sq * sk;
@@ -348,13 +356,38 @@ void sa_oracle_attn_rows(const int8_t *q_i8, const float *q_scale, const int8_t 
     free(blocks); free(s); free(tk); free(acc); free(blk);
 }
 
+void sa_oracle_attn_rows(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                         const float *k_scale, const uint8_t *v_fp8_t, const float *v_scale,
+                         int B, int H, int N, int d, float sm_scale, const uint8_t *mask,
+                         int group, const int64_t *rows, int64_t nrows, float *out)
+{
+    attn_rows_impl(q_i8, q_scale, k_i8, k_scale, v_fp8_t, v_scale, B, H, N, d, sm_scale, mask, group, 0,
+                   rows, nrows, out);
+}
+
+/* Causal quantised attention: as sa_oracle_attn_rows, where row r takes only the keys
+ * t <= r.  Source: "AIGC weekend special 5.10", section 4 (HiAR: every denoising step runs
+ * causal generation over all blocks) and section 6 (SDVG: autoregressive video diffusion):
+ * a query attends to itself and earlier tokens only.
+ * reading: the quantisation is unchanged (scales over all N tokens); the online-softmax
+ * steps are the pairs of kept blocks up to the tile's diagonal pair (2i, 2i+1), and keys
+ * after the row are left out of the step's max and sums. */
+void sa_oracle_attn_rows_causal(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                                const float *k_scale, const uint8_t *v_fp8_t, const float *v_scale,
+                                int B, int H, int N, int d, float sm_scale, const uint8_t *mask,
+                                int group, const int64_t *rows, int64_t nrows, float *out)
+{
+    attn_rows_impl(q_i8, q_scale, k_i8, k_scale, v_fp8_t, v_scale, B, H, N, d, sm_scale, mask, group, 1,
+                   rows, nrows, out);
+}
+
 /* Exact attention in fp64 for selected rows, from the bf16 inputs, with no smoothing
  * and no quantisation: O = softmax(q.K^T * sm_scale) . V over the kept keys (mask
  * semantics as above; NULL = all keys).  out: fp64 [nrows, d]; a row with no kept key
  * gives 0. */
-void sa_oracle_exact_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
-                          int H, int N, int d, double sm_scale, const uint8_t *mask,
-                          const int64_t *rows, int64_t nrows, double *out)
+static void exact_rows_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
+                            int H, int N, int d, double sm_scale, const uint8_t *mask, int causal,
+                            const int64_t *rows, int64_t nrows, double *out)
 {
     (void)B; (void)H;
     const int64_t nq = cdiv64(N, QBLK), nk = cdiv64(N, KBLK);
@@ -367,7 +400,7 @@ void sa_oracle_exact_rows(const uint16_t *q, const uint16_t *k, const uint16_t *
         const uint16_t *vh = v + bh * N * d;
         double mx = -INFINITY;
         for (int64_t t = 0; t < N; ++t) {
-            int keep = !mask || mask[(bh * nq + i) * nk + t / KBLK];
+            int keep = (!mask || mask[(bh * nq + i) * nk + t / KBLK]) && (!causal || t <= r);
             if (!keep) { s[t] = -INFINITY; continue; }
             double acc = 0.0;
             for (int c = 0; c < d; ++c)
@@ -388,6 +421,21 @@ void sa_oracle_exact_rows(const uint16_t *q, const uint16_t *k, const uint16_t *
         for (int c = 0; c < d; ++c) o[c] /= den;
     }
     free(s);
+}
+
+void sa_oracle_exact_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
+                          int H, int N, int d, double sm_scale, const uint8_t *mask,
+                          const int64_t *rows, int64_t nrows, double *out)
+{
+    exact_rows_impl(q, k, v, B, H, N, d, sm_scale, mask, 0, rows, nrows, out);
+}
+
+/* Exact causal attention in fp64: row r over the keys t <= r (and the mask, if any). */
+void sa_oracle_exact_rows_causal(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B,
+                                 int H, int N, int d, double sm_scale, const uint8_t *mask,
+                                 const int64_t *rows, int64_t nrows, double *out)
+{
+    exact_rows_impl(q, k, v, B, H, N, d, sm_scale, mask, 1, rows, nrows, out);
 }
 
 /* int32 S = q_i8 . k_i8^T for selected query rows against all Npad key rows (padded
