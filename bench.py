@@ -225,6 +225,7 @@ def main():
                     help="query rows in the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sla", action="store_true", help="skip the SLA forward timing")
+    ap.add_argument("--no-causal", action="store_true", help="skip the causal forward timing")
     ap.add_argument("--linear-workload", default=DEFAULT_LINEAR, choices=list(LINEAR_WORKLOADS) + ["none"],
                     help="W8A8 linear layer timed beside the attention step ('none' skips it)")
     args = ap.parse_args()
@@ -346,6 +347,29 @@ def main():
 
     peak, peak_src = measured_peak()
 
+    # ---- the causal forward on the same inputs: each 128-query tile visits the 64-key
+    # blocks up to its diagonal pair; ops counted over the blocks executed
+    causal = None
+    if not args.no_causal and w.mask_density is None:
+        nq, nk = -(-w.N // 128), -(-w.N // 64)
+        blocks = sum(min(2 * i + 2, nk) for i in range(nq)) * w.B * w.H
+        ops_causal = 4.0 * 128 * 64 * w.d * blocks
+        for _ in range(args.warmup):
+            sa.sa_attn_fwd_causal(dq, dk, dv, w.sm_scale, out=do)
+        barrier()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            sa.sa_attn_fwd_causal(dq, dk, dv, w.sm_scale, out=do)
+        c1.record(stream)
+        barrier()
+        t_causal = slowest(c0.elapsed_time(c1) / 1e3 / args.steps)
+        assert sa.sa_get_device_status() == 0
+        causal = {"step": "sa_attn_fwd_causal: prologue + masked kernel over the blocks up to the diagonal, "
+                          "keys after each row dropped",
+                  "ms": t_causal * 1e3, "executed_block_fraction": blocks / (w.B * w.H * nq * nk),
+                  "executed_tops": whole_job_tops(ops_causal, world, t_causal)}
+
     # ---- the SLA forward on the same inputs: sparse quantised attention over the critical
     # blocks plus linear attention over the marginal blocks, projected
     sla = None
@@ -454,6 +478,8 @@ def main():
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
         }
+        if causal is not None:
+            line["causal"] = causal
         if sla is not None:
             line["sla"] = sla
         if w8a8 is not None:

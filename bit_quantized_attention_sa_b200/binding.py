@@ -30,6 +30,7 @@ _lib.sa_quantize_qk_noalloc.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, 
 _lib.sa_quantize_v.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
+_lib.sa_attn_fwd_causal.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
 _lib.sa_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
@@ -50,6 +51,7 @@ _lib.sa_release_workspace.argtypes = []
 _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
+              "sa_attn_fwd_causal",
               "sa_attn_fwd_quantized",
               "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_sla_linear", "sa_sla_fwd", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
@@ -165,6 +167,23 @@ def sa_attn_fwd(q, k, v, sm_scale: float | None = None, block_mask=None, out=Non
     _need(o, torch.bfloat16, "out")
     _check(_lib.sa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, float(sm_scale),
                             _ptr(m), _stream(q.device)), "sa_attn_fwd")
+    return o
+
+
+def sa_attn_fwd_causal(q, k, v, sm_scale: float | None = None, block_mask=None, out=None):
+    """Causal forward: query row r attends to the keys t <= r (and the kept blocks of
+    block_mask, if given)."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, name)
+    B, H, N, d = _dims(q)
+    if tuple(k.shape) != (B, H, N, d) or tuple(v.shape) != (B, H, N, d):
+        raise ValueError("q, k and v shapes differ")
+    scale = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device) if out is None else out
+    _need(o, torch.bfloat16, "out")
+    m = _mask_arg(block_mask, B, H, N, q.device)
+    _check(_lib.sa_attn_fwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, scale, _ptr(m),
+                                   _stream(q.device)), "sa_attn_fwd_causal")
     return o
 
 

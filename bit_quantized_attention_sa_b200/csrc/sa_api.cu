@@ -158,7 +158,7 @@ static sa_status get_workspace(size_t bytes, uint8_t **out)
 static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t *k8,
                                 const float *sk, const uint8_t *v8, const float *sv, void *o,
                                 const Shape &s, float sm_scale, const uint8_t *mask,
-                                cudaStream_t st)
+                                cudaStream_t st, bool causal = false)
 {
     AttnArgs a;
     const uint64_t rows = uint64_t(s.BH() * s.Npad());
@@ -178,13 +178,14 @@ static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t 
     a.nq = int(s.nq());
     a.nk = int(s.nk());
     a.sm_scale = sm_scale;
+    a.causal = causal ? 1 : 0;
     return launch_attention(a, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 // Prologue into the library workspace, then the fused attention kernel (validated args).
 static sa_status attn_fwd_device(const void *q, const void *k, const void *v, void *o,
                                  const Shape &s, float sm_scale, const uint8_t *block_mask,
-                                 cudaStream_t st)
+                                 cudaStream_t st, bool causal = false)
 {
     const WsLayout L = ws_layout(s);
     uint8_t *ws = nullptr;
@@ -202,7 +203,7 @@ static sa_status attn_fwd_device(const void *q, const void *k, const void *v, vo
     if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st) !=
         cudaSuccess)
         return SA_ERR_CUDA;
-    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st);
+    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st, causal);
 }
 
 // ------------------------------------------------------------------ host-buffer pipeline
@@ -567,6 +568,24 @@ sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B
                              reinterpret_cast<float *>(ws + attn + mb + sb), true, o, st) == cudaSuccess
                ? SA_OK
                : SA_ERR_CUDA;
+}
+
+sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *o, int B, int H, int N, int d,
+                             float sm_scale, const uint8_t *block_mask, void *stream)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, d, &s);
+    if (r != SA_OK) return r;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
+    if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
+    if ((r = check_device()) != SA_OK) return r;
+    // workspace: [attention prologue | causal block mask]
+    const size_t attn = align256(ws_layout(s).total);
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(attn + size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk()), &ws)) != SA_OK) return r;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_causal_mask(block_mask, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
+    return attn_fwd_device(q, k, v, o, s, sm_scale, ws + attn, st, true);
 }
 
 sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,

@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ q_scale,
                     const float *__restrict__ k_scale, const float *__restrict__ v_scale,
                     const uint8_t *__restrict__ mask, __nv_bfloat16 *__restrict__ out, int BH,
-                    int N, int Npad, int nq, int nk, float sm_scale)
+                    int N, int Npad, int nq, int nk, float sm_scale, int causal)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -336,7 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, ok);
                 const int2 jp = info[st];
                 const int j = ok ? (wg ? jp.y : jp.x) : -1;  // info is only valid once loaded
-                const int nvalid = j >= 0 ? min(64, N - 64 * j) : 0;
+                int nvalid = j >= 0 ? min(64, N - 64 * j) : 0;
+                // causal: row qrow keeps the keys t <= qrow of this block
+                if (causal && j >= 0) nvalid = max(0, min(nvalid, qrow - 64 * j + 1));
                 const uint32_t taddr = tmem + lane_addr + (sb ? kColS1 : kColS0) + 64 * wg;
 
                 // S of this half is read from tensor memory once and kept in registers;
@@ -641,8 +643,9 @@ static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
 {
 #ifndef SA_NO_PAIRS
-    if (!a.mask) return launch_attention_pairs(a, st);
+    if (!a.mask && !a.causal) return launch_attention_pairs(a, st);
 #endif
+    if (a.causal && !a.mask) return cudaErrorInvalidValue;  // causal runs need the block mask
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -660,7 +663,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
     const int grid = ntiles < sms ? ntiles : sms;
     attn_fwd_kernel<<<grid, kThreads, kSmemAlloc, st>>>(a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale,
                                                         a.v_scale, a.mask, a.o, a.BH, a.N, a.Npad,
-                                                        a.nq, a.nk, a.sm_scale);
+                                                        a.nq, a.nk, a.sm_scale, a.causal);
     return cudaGetLastError();
 }
 

@@ -44,6 +44,7 @@ struct AttnArgs {
     __nv_bfloat16 *o;
     int BH, N, Npad, nq, nk;
     float sm_scale;
+    int causal = 0;  // row r keeps only the keys t <= r (mask must then be set)
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
 cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k, int BH,
@@ -54,6 +55,8 @@ cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t
 constexpr int kMaskMaxKeyBlocks = 4096;  // key blocks per mask row the selector sorts in shared memory
 cudaError_t launch_pool_qk(const void *q, const void *k, const Shape &s, float *qbar, float *kbar,
                            cudaStream_t st);
+// Causal block mask: out[bh][i][j] = (j <= 2i + 1) && (user == null || user[bh][i][j] != 0).
+cudaError_t launch_causal_mask(const uint8_t *user, const Shape &s, uint8_t *out, cudaStream_t st);
 cudaError_t launch_block_select(const float *qbar, const float *kbar, double *scores, const Shape &s,
                                 int keep_per_row, int keep_diagonal, uint8_t *mask, cudaStream_t st);
 // ---- W8A8 linear layer (sa_w8a8.cu)

@@ -194,7 +194,26 @@ __global__ void __launch_bounds__(kSelThreads)
     if (keep_diagonal && tid < 2 && 2 * i + tid < nk) mrow[2 * i + tid] = 1;
 }
 
+// grid-stride over BH * nq * nk entries.
+__global__ void causal_mask_kernel(const uint8_t *__restrict__ user, int64_t nq, int64_t nk, int64_t n,
+                                   uint8_t *__restrict__ out)
+{
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t j = e % nk, i = (e / nk) % nq;
+        out[e] = (j <= 2 * i + 1 && (!user || user[e])) ? 1 : 0;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_causal_mask(const uint8_t *user, const Shape &s, uint8_t *out, cudaStream_t st)
+{
+    const int64_t n = s.BH() * s.nq() * s.nk();
+    const int64_t want = (n + 255) / 256;
+    const int blocks = int(want < 4096 ? want : 4096);
+    causal_mask_kernel<<<blocks, 256, 0, st>>>(user, s.nq(), s.nk(), n, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pool_qk(const void *q, const void *k, const Shape &s, float *qbar, float *kbar,
                            cudaStream_t st)

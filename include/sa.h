@@ -110,6 +110,16 @@ sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp
 sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
                       int N, int d, float sm_scale, const uint8_t *block_mask, void *stream);
 
+/* Causal forward: as sa_attn_fwd, where query row r attends to the keys t <= r only.
+ * Source: "AIGC weekend special 5.10", sections 4 (HiAR: causal generation over all blocks
+ * at each denoising step) and 6 (SDVG: autoregressive video diffusion).  Reading: the
+ * quantisation is unchanged (scales over all N tokens); a tile of 128 queries visits its
+ * kept blocks j <= 2i + 1 in pairs, as without causality, and keys after the row are left
+ * out of the max and the sums.  block_mask (or NULL) is intersected with the causal
+ * block pattern.  Uses the library workspace (plus nq * nk bytes per head for the mask). */
+sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *o, int B, int H, int N,
+                             int d, float sm_scale, const uint8_t *block_mask, void *stream);
+
 /* Full forward on HOST buffers: q, k, v, o bf16 [B,H,N,d] and block_mask (or NULL) in host
  * memory, page-locked for the copies to overlap (pageable memory works but serialises).
  * The B*H heads are independent, so they are processed in chunks of consecutive heads:

@@ -99,3 +99,12 @@ def test_sla_argument_errors(libsa):
     assert lib.sa_sla_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, ctypes.c_float(0.0), FAKE, 0, None, None) == 1
     assert lib.sa_sla_fwd(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, f, FAKE, 1, None, None) == 3
     assert lib.sa_sla_fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, f, FAKE, 1, None, None) == 1
+
+
+def test_causal_argument_errors(libsa):
+    lib = libsa.raw_library()
+    f = ctypes.c_float(0.088)
+    assert lib.sa_attn_fwd_causal(None, FAKE, FAKE, FAKE, 1, 1, 128, 128, f, None, None) == 1
+    assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, f, None, None) == 2
+    assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, f, None, None) == 3
+    assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, ctypes.c_float(-1.0), None, None) == 1

@@ -1,0 +1,73 @@
+"""Causal attention on the GPU against the oracle's causal rows: rows on both sides of every
+64-key boundary of the diagonal blocks, ragged tails, a user block mask intersected with the
+causal pattern, the last row against the non-causal masked kernel, and full size at 480p."""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_attention_sa_b200.workloads import WORKLOADS, make_inputs, make_workload
+
+from _helpers import O_MAX_ABS, O_MIN_COS, cosine, gpu_rows, sm_scale, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _boundary_rows(B, H, N):
+    picks = {0, 1, 62, 63, 64, 65, 126, 127, 128, 129, 191, 192, 255, 256, N // 2, N - 2, N - 1}
+    return [(bh, r) for bh in range(B * H) for r in sorted(picks) if 0 <= r < N]
+
+
+def _check(oracle, q, k, v, o, rows, mask=None):
+    B, H, N, _ = q.shape
+    ref = oracle.attn_rows(oracle.quantize_qk(q, k), oracle.quantize_v(v), N, sm_scale(), rows, mask, 2,
+                           causal=True)
+    got = gpu_rows(o, rows)
+    assert np.abs(got - ref).max() <= O_MAX_ABS
+    assert cosine(got, ref) >= O_MIN_COS
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 2, 1), (1, 2, 65), (1, 2, 300), (2, 1, 1000), (1, 2, 3000)])
+def test_causal_matches_oracle(oracle, libsa, cuda_ok, B, H, N):
+    q, k, v, _ = make_inputs(B, H, N, seed=140 + N, outliers=True)
+    o = libsa.sa_attn_fwd_causal(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v))
+    assert libsa.sa_get_device_status() == 0
+    _check(oracle, q, k, v, o, _boundary_rows(B, H, N))
+
+
+def test_last_row_equals_non_causal_masked_kernel(libsa, cuda_ok):
+    """The last row sees every key: the causal run and the masked run with every block kept
+    take the same steps on the same values, bit for bit."""
+    N = 1000
+    q, k, v, _ = make_inputs(1, 2, N, seed=150, outliers=True)
+    qd, kd, vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+    ones = torch.ones((1, 2, -(-N // 128), -(-N // 64)), dtype=torch.uint8, device="cuda")
+    oc = libsa.sa_attn_fwd_causal(qd, kd, vd)
+    om = libsa.sa_attn_fwd(qd, kd, vd, block_mask=ones)
+    assert torch.equal(oc[:, :, N - 1].view(torch.int16), om[:, :, N - 1].view(torch.int16))
+
+
+def test_causal_with_block_mask(oracle, libsa, cuda_ok):
+    B, H, N = 1, 2, 2000
+    q, k, v, _ = make_inputs(B, H, N, seed=151, outliers=True)
+    rng = np.random.default_rng(151)
+    nq, nk = -(-N // 128), -(-N // 64)
+    mask = (rng.random((B, H, nq, nk)) < 0.5).astype(np.uint8)
+    for i in range(nq):
+        mask[:, :, i, 2 * i] = 1  # every row keeps its own first diagonal block
+    o = libsa.sa_attn_fwd_causal(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v),
+                                 block_mask=torch.from_numpy(mask).cuda())
+    assert libsa.sa_get_device_status() == 0
+    _check(oracle, q, k, v, o, _boundary_rows(B, H, N), mask)
+
+
+def test_causal_full_size_480p(oracle, libsa, cuda_ok):
+    w = WORKLOADS["wan14b-480p-h40-n32760"]
+    q, k, v, _ = make_workload(w)
+    o = libsa.sa_attn_fwd_causal(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v), w.sm_scale)
+    assert libsa.sa_get_device_status() == 0
+    rows = [(0, 0), (0, 127), (5, 128), (11, 5000), (23, 16447), (39, 32639), (39, 32640), (17, 32759)]
+    ref = oracle.attn_rows(oracle.quantize_qk(q, k), oracle.quantize_v(v), w.N, w.sm_scale, rows, None, 2,
+                           causal=True)
+    got = gpu_rows(o, rows)
+    assert np.abs(got - ref).max() <= O_MAX_ABS
+    assert cosine(got, ref) >= O_MIN_COS
