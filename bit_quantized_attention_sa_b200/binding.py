@@ -31,6 +31,7 @@ _lib.sa_quantize_v.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_causal.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
+_lib.sa_attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _I, _P, _I, _I, _F, _I, _P]
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
 _lib.sa_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
@@ -51,7 +52,7 @@ _lib.sa_release_workspace.argtypes = []
 _lib.sa_padded_len.argtypes = [_I]
 _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
-              "sa_attn_fwd_causal",
+              "sa_attn_fwd_causal", "sa_attn_fwd_varlen",
               "sa_attn_fwd_quantized",
               "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_sla_linear", "sa_sla_fwd", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
               "sa_release_workspace"):
@@ -184,6 +185,25 @@ def sa_attn_fwd_causal(q, k, v, sm_scale: float | None = None, block_mask=None, 
     m = _mask_arg(block_mask, B, H, N, q.device)
     _check(_lib.sa_attn_fwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, scale, _ptr(m),
                                    _stream(q.device)), "sa_attn_fwd_causal")
+    return o
+
+
+def sa_attn_fwd_varlen(q, k, v, seqlens, H: int, sm_scale: float | None = None, causal: bool = False, out=None):
+    """Packed variable-length batch: q, k, v contiguous bf16 CUDA tensors of H * sum(seqlens)
+    * d elements (any shape; sequence i is its [1, H, N_i, d] block after the earlier
+    sequences').  Returns o of the same shape."""
+    for t, name in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, name)
+    lens = [int(n) for n in seqlens]
+    d = int(q.shape[-1])
+    if q.numel() != H * sum(lens) * d or k.numel() != q.numel() or v.numel() != q.numel():
+        raise ValueError("q, k and v must hold H * sum(seqlens) * d elements")
+    scale = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
+    o = torch.empty_like(q) if out is None else out
+    _need(o, torch.bfloat16, "out")
+    arr = (ctypes.c_int * len(lens))(*lens)
+    _check(_lib.sa_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), len(lens), arr, int(H), d, scale,
+                                   int(bool(causal)), _stream(q.device)), "sa_attn_fwd_varlen")
     return o
 
 

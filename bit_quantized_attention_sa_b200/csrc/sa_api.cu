@@ -588,6 +588,50 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
     return attn_fwd_device(q, k, v, o, s, sm_scale, ws + attn, st, true);
 }
 
+sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int nseq, const int *seqlens,
+                             int H, int d, float sm_scale, int causal, void *stream)
+{
+    if (nseq < 1 || !seqlens || H < 1) return SA_ERR_INVALID_ARG;
+    if (d != kD) return SA_ERR_UNSUPPORTED;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
+    sa_status r = check_ptrs({q, k, v, o});
+    if (r != SA_OK) return r;
+    // validate every sequence and size the workspace for the largest before any launch
+    size_t need = 0;
+    for (int i = 0; i < nseq; ++i) {
+        Shape s;
+        if ((r = check_shape(1, H, seqlens[i], d, &s)) != SA_OK) return r;
+        size_t b = align256(ws_layout(s).total);
+        if (causal) b += size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk());
+        need = std::max(need, b);
+    }
+    if ((r = check_device()) != SA_OK) return r;
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(need, &ws)) != SA_OK) return r;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // sequence i occupies H * N_i * d consecutive elements of each tensor, after those of
+    // the sequences before it; each is an independent [1, H, N_i, d] problem
+    int64_t off = 0;
+    for (int i = 0; i < nseq; ++i) {
+        Shape s;
+        check_shape(1, H, seqlens[i], d, &s);
+        const auto *qi = static_cast<const uint16_t *>(q) + off, *ki = static_cast<const uint16_t *>(k) + off,
+                   *vi = static_cast<const uint16_t *>(v) + off;
+        auto *oi = static_cast<uint16_t *>(o) + off;
+        if ((reinterpret_cast<uintptr_t>(qi) & 15u) != 0) return SA_ERR_MISALIGNED;
+        if (causal) {
+            const size_t attn = align256(ws_layout(s).total);
+            if (launch_causal_mask(nullptr, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
+            r = attn_fwd_device(qi, ki, vi, oi, s, sm_scale, ws + attn, st, true);
+        } else {
+            r = attn_fwd_device(qi, ki, vi, oi, s, sm_scale, nullptr, st);
+        }
+        if (r != SA_OK) return r;
+        off += int64_t(H) * seqlens[i] * kD;
+    }
+    return SA_OK;
+}
+
 sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,
                           int32_t *s_out, void *stream)
 {

@@ -120,6 +120,17 @@ sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int 
 sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *o, int B, int H, int N,
                              int d, float sm_scale, const uint8_t *block_mask, void *stream);
 
+/* Variable-length batch: nseq independent sequences of lengths seqlens[i] (host array,
+ * each >= 1), packed back to back: sequence i is a [1, H, N_i, d] bf16 block of q, k, v
+ * and o starting H * (N_0 + ... + N_{i-1}) * d elements in.  Each sequence is computed as
+ * sa_attn_fwd (causal = 0) or sa_attn_fwd_causal without a mask (causal != 0) would compute
+ * it alone, with the same results.  Every block must start 16-byte aligned (H * N_i * d is a
+ * multiple of 8 elements, which d = 128 guarantees).  All sizes are checked before the first
+ * launch.  The workspace is sized for the largest sequence; the sequences run one after
+ * another on `stream`. */
+sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int nseq, const int *seqlens,
+                             int H, int d, float sm_scale, int causal, void *stream);
+
 /* Full forward on HOST buffers: q, k, v, o bf16 [B,H,N,d] and block_mask (or NULL) in host
  * memory, page-locked for the copies to overlap (pageable memory works but serialises).
  * The B*H heads are independent, so they are processed in chunks of consecutive heads:

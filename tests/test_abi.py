@@ -108,3 +108,15 @@ def test_causal_argument_errors(libsa):
     assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, f, None, None) == 2
     assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, f, None, None) == 3
     assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, ctypes.c_float(-1.0), None, None) == 1
+
+
+def test_varlen_argument_errors(libsa):
+    lib = libsa.raw_library()
+    f = ctypes.c_float(0.088)
+    lens = (ctypes.c_int * 3)(100, 0, 50)
+    ok = (ctypes.c_int * 2)(100, 50)
+    assert lib.sa_attn_fwd_varlen(FAKE, FAKE, FAKE, FAKE, 0, ok, 2, 128, f, 0, None) == 1
+    assert lib.sa_attn_fwd_varlen(FAKE, FAKE, FAKE, FAKE, 2, None, 2, 128, f, 0, None) == 1
+    assert lib.sa_attn_fwd_varlen(FAKE, FAKE, FAKE, FAKE, 3, lens, 2, 128, f, 0, None) == 1   # N = 0
+    assert lib.sa_attn_fwd_varlen(FAKE, FAKE, FAKE, FAKE, 2, ok, 2, 64, f, 0, None) == 2
+    assert lib.sa_attn_fwd_varlen(FAKE, FAKE, FAKE, ODD, 2, ok, 2, 128, f, 1, None) == 3

@@ -1,0 +1,38 @@
+"""The packed variable-length entry point: each sequence of the batch comes out bit for bit
+as its own sa_attn_fwd (or sa_attn_fwd_causal) call, for ragged lengths including 1, 64 and
+non-multiples of 128, and a sampled row matches the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from bit_quantized_attention_sa_b200.workloads import make_inputs
+
+from _helpers import O_MAX_ABS, O_MIN_COS, cosine, sm_scale, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_equals_per_sequence_calls(oracle, libsa, cuda_ok, causal):
+    H, lens = 2, [1, 200, 129, 1000, 64, 333]
+    seqs = [make_inputs(1, H, n, seed=160 + n, outliers=True)[:3] for n in lens]
+    packed = [torch.cat([to_dev_bf16(s[t]).reshape(-1) for s in seqs]) for t in range(3)]
+    o = libsa.sa_attn_fwd_varlen(*packed, lens, H, causal=causal)
+    assert libsa.sa_get_device_status() == 0
+    off = 0
+    for n, (q, k, v) in zip(lens, seqs):
+        qd, kd, vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+        ref = libsa.sa_attn_fwd_causal(qd, kd, vd) if causal else libsa.sa_attn_fwd(qd, kd, vd)
+        got = o[off:off + H * n * 128].reshape(1, H, n, 128)
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), n
+        off += H * n * 128
+    # one sequence against the oracle
+    q, k, v = seqs[3]
+    rows = [(bh, r) for bh in range(H) for r in (0, 127, 128, 640, 999)]
+    start = H * (lens[0] + lens[1] + lens[2]) * 128
+    blk = o[start:start + H * 1000 * 128].reshape(H, 1000, 128).float().cpu().numpy()
+    got = np.stack([blk[bh, r] for bh, r in rows])
+    ref = oracle.attn_rows(oracle.quantize_qk(q, k), oracle.quantize_v(v), 1000, sm_scale(), rows, None, 2,
+                           causal=causal)
+    assert np.abs(got - ref).max() <= O_MAX_ABS
+    assert cosine(got, ref) >= O_MIN_COS
