@@ -188,14 +188,15 @@ def sa_attn_fwd_causal(q, k, v, sm_scale: float | None = None, block_mask=None, 
     return o
 
 
-def sa_attn_fwd_varlen(q, k, v, seqlens, H: int, sm_scale: float | None = None, causal: bool = False, out=None):
+def sa_attn_fwd_varlen(q, k, v, seqlens, H: int, sm_scale: float | None = None, causal: bool = False, out=None,
+                       d: int = 128):
     """Packed variable-length batch: q, k, v contiguous bf16 CUDA tensors of H * sum(seqlens)
     * d elements (any shape; sequence i is its [1, H, N_i, d] block after the earlier
     sequences').  Returns o of the same shape."""
     for t, name in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, torch.bfloat16, name)
     lens = [int(n) for n in seqlens]
-    d = int(q.shape[-1])
+    d = int(d)
     if q.numel() != H * sum(lens) * d or k.numel() != q.numel() or v.numel() != q.numel():
         raise ValueError("q, k and v must hold H * sum(seqlens) * d elements")
     scale = 1.0 / math.sqrt(d) if sm_scale is None else float(sm_scale)
