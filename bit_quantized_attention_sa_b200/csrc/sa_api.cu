@@ -377,9 +377,57 @@ sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp
     return e == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
+// d = 64: the inputs are zero-padded to 128 channels in the workspace (after the d = 128
+// call's own region, `inner` bytes), the d = 128 path runs on them, and O's first 64
+// channels are copied out.  Zero channels add nothing to S, leave every block maximum (and
+// so every scale and code) unchanged, have mean 0 and V scale 0: the result is the d = 64
+// definition's.  The kernel's time is set by the softmax per score, not by d.
+static sa_status attn_fwd_d64(const void *q, const void *k, const void *v, void *o, int B, int H, int N,
+                              float sm_scale, const uint8_t *block_mask, bool causal, cudaStream_t st)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, kD, &s);
+    if (r != SA_OK) return r;
+    size_t inner = align256(ws_layout(s).total);
+    if (causal) inner = align256(inner + size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk()));
+    const int64_t rows = s.BH() * s.N;
+    const size_t tb = align256(size_t(rows) * kD * 2);
+    uint8_t *ws = nullptr;
+    if ((r = get_workspace(inner + 4 * tb, &ws)) != SA_OK) return r;
+    uint8_t *pq = ws + inner, *pk = pq + tb, *pv = pk + tb, *po = pv + tb;
+    if (launch_pad_heads(q, rows, pq, st) != cudaSuccess || launch_pad_heads(k, rows, pk, st) != cudaSuccess ||
+        launch_pad_heads(v, rows, pv, st) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (causal) {
+        const size_t attn = align256(ws_layout(s).total);
+        if (launch_causal_mask(block_mask, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
+        r = attn_fwd_device(pq, pk, pv, po, s, sm_scale, ws + attn, st, true);
+    } else {
+        r = attn_fwd_device(pq, pk, pv, po, s, sm_scale, block_mask, st);
+    }
+    if (r != SA_OK) return r;
+    return launch_unpad_heads(po, rows, o, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+static sa_status check_d64_call(int B, int H, int N, float sm_scale, std::initializer_list<const void *> ptrs)
+{
+    Shape s;
+    sa_status r = check_shape(B, H, N, kD, &s);
+    if (r != SA_OK) return r;
+    if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
+    if ((r = check_ptrs(ptrs)) != SA_OK) return r;
+    return check_device();
+}
+
 sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int B, int H,
                       int N, int d, float sm_scale, const uint8_t *block_mask, void *stream)
 {
+    if (d == kD / 2) {
+        const sa_status r = check_d64_call(B, H, N, sm_scale, {q, k, v, o});
+        return r != SA_OK ? r
+                          : attn_fwd_d64(q, k, v, o, B, H, N, sm_scale, block_mask, false,
+                                         static_cast<cudaStream_t>(stream));
+    }
     Shape s;
     sa_status r = check_shape(B, H, N, d, &s);
     if (r != SA_OK) return r;
@@ -573,6 +621,12 @@ sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B
 sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *o, int B, int H, int N, int d,
                              float sm_scale, const uint8_t *block_mask, void *stream)
 {
+    if (d == kD / 2) {
+        const sa_status r = check_d64_call(B, H, N, sm_scale, {q, k, v, o});
+        return r != SA_OK ? r
+                          : attn_fwd_d64(q, k, v, o, B, H, N, sm_scale, block_mask, true,
+                                         static_cast<cudaStream_t>(stream));
+    }
     Shape s;
     sa_status r = check_shape(B, H, N, d, &s);
     if (r != SA_OK) return r;

@@ -32,6 +32,9 @@ cudaError_t launch_quantize_qk(const void *q, const void *k, const Shape &s, int
                                double *k_partial /* [BH, nchunks, d] */, cudaStream_t st);
 cudaError_t launch_quantize_v(const void *v, const Shape &s, uint8_t *v_t, float *v_scale,
                               uint32_t *v_amax_bits /* [BH, d] */, cudaStream_t st);
+// d = 64 calls: [rows][64] bf16 -> [rows][128] with zero upper channels, and back.
+cudaError_t launch_pad_heads(const void *src, int64_t rows, void *dst, cudaStream_t st);
+cudaError_t launch_unpad_heads(const void *src, int64_t rows, void *dst, cudaStream_t st);
 // Fixed scratch for the allocation-free Q/K quantisation: [BH, nchunks, d] fp64 must fit.
 constexpr size_t kNoAllocPartialDoubles = (size_t(4) << 20) / sizeof(double);  // 4 MiB
 cudaError_t noalloc_kpart(double **out);

@@ -274,7 +274,46 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// Head-size padding for d = 64 calls: rows of 64 bf16 channels <-> rows of 128 whose upper
+// 64 channels are zero.  One thread per 16-byte group (8 channels) of the wider row.
+__global__ void pad_heads_kernel(const uint4 *__restrict__ src, int64_t rows, uint4 *__restrict__ dst)
+{
+    const int64_t n = rows * 16;
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = e >> 4;
+        const int g = int(e & 15);
+        dst[e] = g < 8 ? src[r * 8 + g] : make_uint4(0, 0, 0, 0);
+    }
+}
+
+__global__ void unpad_heads_kernel(const uint4 *__restrict__ src, int64_t rows, uint4 *__restrict__ dst)
+{
+    const int64_t n = rows * 8;
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x)
+        dst[e] = src[(e >> 3) * 16 + (e & 7)];
+}
+
 }  // namespace
+
+static int grid_for(int64_t n)
+{
+    const int64_t want = (n + 255) / 256;
+    return int(want < 8192 ? want : 8192);
+}
+
+cudaError_t launch_pad_heads(const void *src, int64_t rows, void *dst, cudaStream_t st)
+{
+    pad_heads_kernel<<<grid_for(rows * 16), 256, 0, st>>>(static_cast<const uint4 *>(src), rows,
+                                                         static_cast<uint4 *>(dst));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpad_heads(const void *src, int64_t rows, void *dst, cudaStream_t st)
+{
+    unpad_heads_kernel<<<grid_for(rows * 8), 256, 0, st>>>(static_cast<const uint4 *>(src), rows,
+                                                          static_cast<uint4 *>(dst));
+    return cudaGetLastError();
+}
 
 // Scratch of sa_quantize_qk_noalloc: the fp64 per-chunk column sums of K, in a fixed
 // device array instead of the library's cudaMalloc'd workspace.  It lives for the whole

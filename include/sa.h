@@ -27,7 +27,10 @@
  *   O = acc * scale_v / l (bf16), 0 for a row with no kept key.
  *
  * Conventions for every entry point:
- *   - Tensors are contiguous row-major.  q, k, v, o: bf16 [B,H,N,d].  d must be 128.
+ *   - Tensors are contiguous row-major.  q, k, v, o: bf16 [B,H,N,d].  d must be 128, except
+ *     that sa_attn_fwd and sa_attn_fwd_causal also take d = 64: they zero-pad q, k, v to 128
+ *     channels in the workspace and copy out o's first 64, which gives exactly the d = 64
+ *     definition (zero channels add nothing to S and leave every scale and code unchanged).
  *     Npad = 128 * ceil(N/128); nq = ceil(N/128); nk = ceil(N/64).
  *   - Device pointers are owned by the caller; the library never frees them.  All
  *     pointers must be 16-byte aligned.

@@ -39,7 +39,7 @@ ODD = ctypes.c_void_p((1 << 20) + 8)  # misaligned
 
 @pytest.mark.parametrize("args,expect", [
     ((None, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0.088, None, None), 1),   # null q
-    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0.088, None, None), 2),    # d != 128
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, 0.088, None, None), 2),    # d not 64 or 128
     ((FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, 0.088, None, None), 3),    # misaligned o
     ((FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 0.088, None, None), 1),     # N = 0
     ((FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, 0.088, None, None), 1),   # B = 0
@@ -105,7 +105,12 @@ def test_causal_argument_errors(libsa):
     lib = libsa.raw_library()
     f = ctypes.c_float(0.088)
     assert lib.sa_attn_fwd_causal(None, FAKE, FAKE, FAKE, 1, 1, 128, 128, f, None, None) == 1
-    assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, f, None, None) == 2
+    assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 96, f, None, None) == 2
+    # d = 64 is accepted by the forward calls (zero-padded to 128) but not by the others
+    assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 64, f, None, None) == 3
+    assert lib.sa_attn_fwd(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 64, f, None, None) == 3
+    assert lib.sa_attn_fwd(FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 64, f, None, None) == 1
+    assert lib.sa_quantize_qk(FAKE, FAKE, 1, 1, 128, 64, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2
     assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, ODD, 1, 1, 128, 128, f, None, None) == 3
     assert lib.sa_attn_fwd_causal(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, ctypes.c_float(-1.0), None, None) == 1
 
