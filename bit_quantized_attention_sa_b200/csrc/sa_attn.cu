@@ -642,9 +642,7 @@ static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
 {
-#ifndef SA_NO_PAIRS
     if (!a.mask && !a.causal) return launch_attention_pairs(a, st);
-#endif
     if (a.causal && !a.mask) return cudaErrorInvalidValue;  // causal runs need the block mask
     static bool attr_set[64] = {false};
     int dev = 0;
