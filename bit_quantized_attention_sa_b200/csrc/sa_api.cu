@@ -398,10 +398,12 @@ static sa_status attn_fwd_d64(const void *q, const void *k, const void *v, void 
     if (launch_pad_heads(q, rows, pq, st) != cudaSuccess || launch_pad_heads(k, rows, pk, st) != cudaSuccess ||
         launch_pad_heads(v, rows, pv, st) != cudaSuccess)
         return SA_ERR_CUDA;
-    if (causal) {
+    if (causal && block_mask) {
         const size_t attn = align256(ws_layout(s).total);
         if (launch_causal_mask(block_mask, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
         r = attn_fwd_device(pq, pk, pv, po, s, sm_scale, ws + attn, st, true);
+    } else if (causal) {
+        r = attn_fwd_device(pq, pk, pv, po, s, sm_scale, nullptr, st, true);
     } else {
         r = attn_fwd_device(pq, pk, pv, po, s, sm_scale, block_mask, st);
     }
@@ -633,11 +635,13 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
-    // workspace: [attention prologue | causal block mask]
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // without a keep mask the pair kernel runs the causal pattern itself
+    if (!block_mask) return attn_fwd_device(q, k, v, o, s, sm_scale, nullptr, st, true);
+    // with one: workspace [attention prologue | keep mask intersected with the causal blocks]
     const size_t attn = align256(ws_layout(s).total);
     uint8_t *ws = nullptr;
     if ((r = get_workspace(attn + size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk()), &ws)) != SA_OK) return r;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (launch_causal_mask(block_mask, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
     return attn_fwd_device(q, k, v, o, s, sm_scale, ws + attn, st, true);
 }
@@ -655,9 +659,7 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
     for (int i = 0; i < nseq; ++i) {
         Shape s;
         if ((r = check_shape(1, H, seqlens[i], d, &s)) != SA_OK) return r;
-        size_t b = align256(ws_layout(s).total);
-        if (causal) b += size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk());
-        need = std::max(need, b);
+        need = std::max(need, align256(ws_layout(s).total));
     }
     if ((r = check_device()) != SA_OK) return r;
     uint8_t *ws = nullptr;
@@ -673,13 +675,7 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
                    *vi = static_cast<const uint16_t *>(v) + off;
         auto *oi = static_cast<uint16_t *>(o) + off;
         if ((reinterpret_cast<uintptr_t>(qi) & 15u) != 0) return SA_ERR_MISALIGNED;
-        if (causal) {
-            const size_t attn = align256(ws_layout(s).total);
-            if (launch_causal_mask(nullptr, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
-            r = attn_fwd_device(qi, ki, vi, oi, s, sm_scale, ws + attn, st, true);
-        } else {
-            r = attn_fwd_device(qi, ki, vi, oi, s, sm_scale, nullptr, st);
-        }
+        r = attn_fwd_device(qi, ki, vi, oi, s, sm_scale, nullptr, st, causal != 0);
         if (r != SA_OK) return r;
         off += int64_t(H) * seqlens[i] * kD;
     }

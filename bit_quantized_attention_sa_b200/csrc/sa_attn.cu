@@ -636,14 +636,14 @@ static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)
     const int grid = npairs < sms ? npairs : sms;
     attn_pairs_kernel<<<grid, pairs::kThreads, pairs::kSmemAlloc, st>>>(
         a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale, a.v_scale, a.o, a.BH, a.N, a.Npad, a.nq, a.nk,
-        a.sm_scale);
+        a.sm_scale, a.causal);
     return cudaGetLastError();
 }
 
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
 {
-    if (!a.mask && !a.causal) return launch_attention_pairs(a, st);
-    if (a.causal && !a.mask) return cudaErrorInvalidValue;  // causal runs need the block mask
+    // without a keep mask (causal or not): two query tiles per CTA
+    if (!a.mask) return launch_attention_pairs(a, st);
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ q_scale,
                       const float *__restrict__ k_scale, const float *__restrict__ v_scale,
                       __nv_bfloat16 *__restrict__ out, int BH, int N, int Npad, int nq, int nk,
-                      float sm_scale)
+                      float sm_scale, int causal)
 {
     using pairs::kStages;
     using pairs::kThreads;
@@ -240,6 +240,11 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
     const int npairs_h = (nq + 1) / 2, npairs = BH * npairs_h;
     const int nsteps = (nk + 1) / 2;  // every block kept: blocks 2j and 2j+1 form step j
     const bool odd_tail = (nk & 1) != 0;  // the last step then has one block
+    // causal: the pair (qa, qa + 1) needs the steps up to tile qa + 1's diagonal, qa + 2 of
+    // them (qa + 1 for a lone last tile); tile qa's last step is then fully masked
+    auto pair_steps = [&](int qa) -> int {
+        return causal ? min(nsteps, qa + (qa + 1 < nq ? 2 : 1)) : nsteps;
+    };
 
     if (warp >= kWarpProducer) {
         setmaxnreg_dec<kRegsCtrl>();
@@ -257,7 +262,8 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                     if (hasb)
                         tma_load_2d(sbase + kOffQ + kQTileBytes, &tm_q, bar(kBarQFull), 0, bh * Npad + qa * 128 + 128);
                 }
-                for (int j = 0; j < nsteps && ok; ++j, ++g) {
+                const int ns = pair_steps(qa);
+                for (int j = 0; j < ns && ok; ++j, ++g) {
                     const uint32_t st = g % kStages;
                     const bool two = !(odd_tail && j == nsteps - 1);
                     if (g >= kStages) ok = mbar_wait(bar(kBarKvEmpty + st), ((g / kStages) - 1) & 1, abort_flag);
@@ -284,7 +290,8 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                 const int ntile = qa + 1 < nq ? 2 : 1;
                 ok = mbar_wait(bar(kBarQFull), pl & 1, abort_flag);
                 tc_fence_after();
-                for (int j = 0; j < nsteps && ok; ++j, ++g) {
+                const int ns = pair_steps(qa);
+                for (int j = 0; j < ns && ok; ++j, ++g) {
                     const uint32_t st = g % kStages;
                     ok = mbar_wait(bar(kBarKvFull + st), (g / kStages) & 1, abort_flag);
                     const uint32_t kb = sbase + kOffK + st * kKTileBytes;
@@ -310,7 +317,8 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             for (int p = blockIdx.x; p < npairs && ok; p += gridDim.x) {
                 const int qa = 2 * (p % npairs_h);
                 const int ntile = qa + 1 < nq ? 2 : 1;
-                for (int j = 0; j < nsteps && ok; ++j, ++g) {
+                const int ns = pair_steps(qa);
+                for (int j = 0; j < ns && ok; ++j, ++g) {
                     const uint32_t st = g % kStages;
                     const int nkk = (odd_tail && j == nsteps - 1) ? 2 : 4;  // K = 64 or 128 keys
                     ok = mbar_wait(bar(kBarKvFull + st), (g / kStages) & 1, abort_flag);
@@ -358,10 +366,16 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             const float sq = q_scale[int64_t(bh) * nq + qt];
             const float *ksrow = k_scale + int64_t(bh) * nk;
             float m = -INFINITY;
-            for (int j = 0; j < nsteps; ++j, ++c) {
+            const int ns = pair_steps(qt - t);
+            for (int j = 0; j < ns; ++j, ++c) {
                 const bool two = !(odd_tail && j == nsteps - 1);
                 const float ks0 = ksrow[2 * j], ks1 = two ? ksrow[2 * j + 1] : 0.0f;
-                const int nv0 = min(64, N - 128 * j), nv1 = two ? min(64, N - 128 * j - 64) : 0;
+                int nv0 = min(64, N - 128 * j), nv1 = two ? min(64, N - 128 * j - 64) : 0;
+                if (causal) {
+                    // this row keeps the keys up to itself
+                    nv0 = max(0, min(nv0, qrow - 128 * j + 1));
+                    nv1 = max(0, min(nv1, qrow - 128 * j - 63));
+                }
                 if (ok) ok = mbar_wait(bar(kBarSFull + t), c & 1, abort_flag);
                 ok = __all_sync(0xffffffffu, ok);
 

@@ -34,16 +34,20 @@ def test_causal_matches_oracle(oracle, libsa, cuda_ok, B, H, N):
     _check(oracle, q, k, v, o, _boundary_rows(B, H, N))
 
 
-def test_last_row_equals_non_causal_masked_kernel(libsa, cuda_ok):
-    """The last row sees every key: the causal run and the masked run with every block kept
-    take the same steps on the same values, bit for bit."""
-    N = 1000
-    q, k, v, _ = make_inputs(1, 2, N, seed=150, outliers=True)
+@pytest.mark.parametrize("N", [1000, 1024, 1100])
+def test_last_row_equals_non_causal(libsa, cuda_ok, N):
+    """The last row sees every key: the causal run takes the same steps on the same values as
+    the non-causal one, bit for bit, both without a mask (the two-tile kernel) and with every
+    block kept (the masked kernel)."""
+    q, k, v, _ = make_inputs(1, 2, N, seed=150 + N, outliers=True)
     qd, kd, vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
     ones = torch.ones((1, 2, -(-N // 128), -(-N // 64)), dtype=torch.uint8, device="cuda")
     oc = libsa.sa_attn_fwd_causal(qd, kd, vd)
+    od = libsa.sa_attn_fwd(qd, kd, vd)
+    assert torch.equal(oc[:, :, N - 1].view(torch.int16), od[:, :, N - 1].view(torch.int16))
+    ocm = libsa.sa_attn_fwd_causal(qd, kd, vd, block_mask=ones)
     om = libsa.sa_attn_fwd(qd, kd, vd, block_mask=ones)
-    assert torch.equal(oc[:, :, N - 1].view(torch.int16), om[:, :, N - 1].view(torch.int16))
+    assert torch.equal(ocm[:, :, N - 1].view(torch.int16), om[:, :, N - 1].view(torch.int16))
 
 
 def test_causal_with_block_mask(oracle, libsa, cuda_ok):
