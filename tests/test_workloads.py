@@ -53,3 +53,38 @@ def test_named_workloads():
     assert [w.H for w in WORKLOADS.values()] == [2, 12, 40, 40, 40]
     w = WORKLOADS["wan14b-720p-h40-n75600"]
     assert abs(w.dense_ops - 1.1705e14) / 1.1705e14 < 1e-3
+
+
+def test_sla_classes_recipe():
+    from bit_quantized_attention_sa_b200.workloads import make_sla_classes
+    a = make_sla_classes(1, 3, 5000, 0.1, 0.4, seed=3)
+    assert np.array_equal(a, make_sla_classes(1, 3, 5000, 0.1, 0.4, seed=3))
+    nq, nk = -(-5000 // 128), -(-5000 // 64)
+    assert a.shape == (1, 3, nq, nk) and a.dtype == np.uint8
+    assert set(np.unique(a)) <= {0, 1, 2}
+    for i in range(nq):  # diagonal blocks are always critical
+        for j in (2 * i, 2 * i + 1):
+            if j < nk:
+                assert (a[:, :, i, j] == 2).all()
+    off = np.ones(a.shape, bool)
+    for i in range(nq):
+        off[:, :, i, 2 * i:2 * i + 2] = False
+    frac = [(a[off] == c).mean() for c in (2, 1, 0)]
+    assert abs(frac[0] - 0.1) < 0.02 and abs(frac[1] - 0.4) < 0.03 and abs(frac[2] - 0.5) < 0.03
+
+
+def test_linear_inputs_recipe():
+    from bit_quantized_attention_sa_b200.workloads import make_linear_inputs
+    x, w = make_linear_inputs(5000, 64, 512, seed=4)
+    x2, w2 = make_linear_inputs(5000, 64, 512, seed=4)
+    assert np.array_equal(x, x2) and np.array_equal(w, w2)
+    assert x.shape == (5000, 512) and w.shape == (64, 512) and x.dtype == np.uint16
+    xf, wf = bf16_bits_to_f32(x), bf16_bits_to_f32(w)
+    # round(1 % of 512) = 5 activation channels scaled by 8; the rest ~ N(0, 1)
+    std = xf.std(axis=0)
+    assert (std > 4).sum() == 5 and abs(np.median(std) - 1.0) < 0.05
+    assert abs(wf.std() * np.sqrt(512) - 1.0) < 0.05
+    # chunked draws (4096 rows at a time) continue one stream: rows past 4096 differ from
+    # the first rows and keep the same statistics
+    assert not np.array_equal(x[:100], x[4096:4196])
+    assert abs(xf[4096:].std(axis=0)[std < 4].mean() - 1.0) < 0.05
