@@ -748,8 +748,10 @@ const char *sa_status_string(sa_status s)
 size_t sa_workspace_bytes(int B, int H, int N, int d)
 {
     Shape s;
-    if (check_shape(B, H, N, d, &s) != SA_OK) return 0;
-    return ws_layout(s).total;
+    if (check_shape(B, H, N, d == kD / 2 ? kD : d, &s) != SA_OK) return 0;
+    if (d != kD / 2) return ws_layout(s).total;
+    // d = 64: the d = 128 workspace, then the four zero-padded copies of q, k, v and o
+    return align256(ws_layout(s).total) + 4 * align256(size_t(s.BH()) * size_t(s.N) * kD * 2);
 }
 
 sa_status sa_release_workspace(void)

@@ -259,7 +259,8 @@ sa_status sa_get_device_status(void);
 /* Human-readable name of a status code (static string). */
 const char *sa_status_string(sa_status s);
 
-/* Bytes of library workspace sa_attn_fwd needs for this problem size (0 on bad sizes). */
+/* Bytes of library workspace sa_attn_fwd needs for this problem size, d = 128 or 64 (0 on
+ * bad sizes).  Causal calls with a keep mask add B * H * ceil(N/128) * ceil(N/64) bytes. */
 size_t sa_workspace_bytes(int B, int H, int N, int d);
 
 /* Frees the current device's workspace (synchronises the device first). */

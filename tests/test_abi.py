@@ -27,7 +27,9 @@ def test_status_strings_and_sizes(libsa):
     assert libsa.sa_status_string(0) == "SA_OK"
     assert libsa.sa_status_string(6) == "SA_ERR_DEVICE_TIMEOUT"
     assert [libsa.padded_len(n) for n in (0, 1, 128, 129, 75600)] == [0, 128, 128, 256, 75648]
-    assert libsa.sa_workspace_bytes(1, 2, 1024, 64) == 0
+    assert libsa.sa_workspace_bytes(1, 2, 1024, 96) == 0
+    # d = 64: the d = 128 workspace plus four zero-padded 128-channel copies
+    assert libsa.sa_workspace_bytes(1, 2, 1024, 64) >= libsa.sa_workspace_bytes(1, 2, 1024, 128) + 4 * 2 * 1024 * 128 * 2
     assert libsa.sa_workspace_bytes(1, 2, 0, 128) == 0
     ws = libsa.sa_workspace_bytes(1, 40, 75600, 128)
     assert 3 * 40 * 75648 * 128 <= ws < 3 * 40 * 75648 * 128 + (1 << 24)
