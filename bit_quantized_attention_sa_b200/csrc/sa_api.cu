@@ -127,18 +127,22 @@ struct DeviceWs {
     size_t bytes = 0;
 };
 static DeviceWs g_ws[64];
-static std::mutex g_ws_mutex;
+// Held by a call from its workspace request until its launches are enqueued, so that no
+// other host thread can grow (and so free) the buffer in between.  Recursive: the d = 64
+// and SLA paths request the workspace again inside the same call.
+static std::recursive_mutex g_ws_mutex;
+typedef std::unique_lock<std::recursive_mutex> WsLock;
 
-// Returns the current device's workspace grown to at least `bytes`.
-static sa_status get_workspace(size_t bytes, uint8_t **out)
+// Returns the current device's workspace grown to at least `bytes`, with `lock` held.
+static sa_status get_workspace(WsLock &lock, size_t bytes, uint8_t **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    if (!lock.owns_lock()) lock = WsLock(g_ws_mutex);
     DeviceWs &w = g_ws[dev];
     if (w.bytes < bytes) {
         if (w.ptr) {
-            // earlier work on any stream may still use the old buffer
+            // work enqueued earlier, on any stream, may still use the old buffer
             if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;
             cudaFree(w.ptr);
             w.ptr = nullptr;
@@ -158,7 +162,7 @@ static sa_status get_workspace(size_t bytes, uint8_t **out)
 static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t *k8,
                                 const float *sk, const uint8_t *v8, const float *sv, void *o,
                                 const Shape &s, float sm_scale, const uint8_t *mask,
-                                cudaStream_t st, bool causal = false)
+                                cudaStream_t st, bool causal = false, const float *addend = nullptr)
 {
     AttnArgs a;
     const uint64_t rows = uint64_t(s.BH() * s.Npad());
@@ -179,17 +183,19 @@ static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t 
     a.nk = int(s.nk());
     a.sm_scale = sm_scale;
     a.causal = causal ? 1 : 0;
+    a.addend = addend;
     return launch_attention(a, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 // Prologue into the library workspace, then the fused attention kernel (validated args).
 static sa_status attn_fwd_device(const void *q, const void *k, const void *v, void *o,
                                  const Shape &s, float sm_scale, const uint8_t *block_mask,
-                                 cudaStream_t st, bool causal = false)
+                                 cudaStream_t st, bool causal = false, const float *addend = nullptr)
 {
     const WsLayout L = ws_layout(s);
+    WsLock lock;
     uint8_t *ws = nullptr;
-    sa_status r = get_workspace(L.total, &ws);
+    sa_status r = get_workspace(lock, L.total, &ws);
     if (r != SA_OK) return r;
     int8_t *q8 = reinterpret_cast<int8_t *>(ws + L.q8);
     int8_t *k8 = reinterpret_cast<int8_t *>(ws + L.k8);
@@ -203,7 +209,7 @@ static sa_status attn_fwd_device(const void *q, const void *k, const void *v, vo
     if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st) !=
         cudaSuccess)
         return SA_ERR_CUDA;
-    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st, causal);
+    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st, causal, addend);
 }
 
 // ------------------------------------------------------------------ host-buffer pipeline
@@ -335,8 +341,9 @@ sa_status sa_quantize_qk(const void *q, const void *k, int B, int H, int N, int 
     if ((r = check_ptrs({q, k, q_i8, q_scale, k_i8, k_scale, k_mean})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     const WsLayout L = ws_layout(s);
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(L.total, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, L.total, &ws)) != SA_OK) return r;
     cudaError_t e = launch_quantize_qk(q, k, s, q_i8, q_scale, k_i8, k_scale, k_mean,
                                        reinterpret_cast<double *>(ws + L.kpart),
                                        static_cast<cudaStream_t>(stream));
@@ -369,8 +376,9 @@ sa_status sa_quantize_v(const void *v, int B, int H, int N, int d, uint8_t *v_fp
     if ((r = check_ptrs({v, v_fp8_t, v_scale})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     const WsLayout L = ws_layout(s);
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(L.total, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, L.total, &ws)) != SA_OK) return r;
     cudaError_t e = launch_quantize_v(v, s, v_fp8_t, v_scale,
                                       reinterpret_cast<uint32_t *>(ws + L.vamax),
                                       static_cast<cudaStream_t>(stream));
@@ -392,8 +400,9 @@ static sa_status attn_fwd_d64(const void *q, const void *k, const void *v, void 
     if (causal) inner = align256(inner + size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk()));
     const int64_t rows = s.BH() * s.N;
     const size_t tb = align256(size_t(rows) * kD * 2);
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(inner + 4 * tb, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, inner + 4 * tb, &ws)) != SA_OK) return r;
     uint8_t *pq = ws + inner, *pk = pq + tb, *pv = pk + tb, *po = pv + tb;
     if (launch_pad_heads(q, rows, pq, st) != cudaSuccess || launch_pad_heads(k, rows, pk, st) != cudaSuccess ||
         launch_pad_heads(v, rows, pv, st) != cudaSuccess)
@@ -480,8 +489,9 @@ sa_status sa_block_mask(const void *q, const void *k, int B, int H, int N, int d
     if ((r = check_device()) != SA_OK) return r;
     const size_t qb = align256(size_t(s.BH() * s.nq()) * kD * 4), kb = align256(size_t(s.BH() * s.nk()) * kD * 4);
     const size_t sb = size_t(s.BH() * s.nq()) * size_t(s.nk()) * 8;
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(qb + kb + sb, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, qb + kb + sb, &ws)) != SA_OK) return r;
     float *qbar = reinterpret_cast<float *>(ws), *kbar = reinterpret_cast<float *>(ws + qb);
     double *scores = reinterpret_cast<double *>(ws + qb + kb);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -558,8 +568,9 @@ sa_status sa_w8a8_linear(const void *x, const int8_t *w_codes, const float *w_sc
     if ((r = check_device()) != SA_OK) return r;
     const size_t kpad = size_t(cdiv(K, 128)) * 128;
     const size_t cb = align256(size_t(M) * kpad), sb = size_t(cdiv(M, 128)) * size_t(kpad / 128) * 4;
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(cb + sb, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, cb + sb, &ws)) != SA_OK) return r;
     int8_t *xc = reinterpret_cast<int8_t *>(ws);
     float *xs = reinterpret_cast<float *>(ws + cb);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -585,11 +596,11 @@ sa_status sa_sla_linear(const void *q, const void *k, const void *v, const uint8
     if (proj && (r = check_ptrs({proj})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     const size_t sb = align256(sla_state_bytes(s));
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(sb + sla_sum_bytes(s), &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, sb + sla_sum_bytes(s), &ws)) != SA_OK) return r;
     return launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws),
-                             reinterpret_cast<float *>(ws + sb), false, out,
-                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+                             reinterpret_cast<float *>(ws + sb), out, static_cast<cudaStream_t>(stream)) == cudaSuccess
                ? SA_OK
                : SA_ERR_CUDA;
 }
@@ -604,20 +615,24 @@ sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B
     if ((r = check_sla(s, phi, {q, k, v, o})) != SA_OK) return r;
     if (proj && (r = check_ptrs({proj})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
-    // workspace: [attention prologue | keep mask | states | summed states]
+    // workspace: [attention prologue | keep mask | states | summed states | linear part, fp32]
     const size_t attn = align256(ws_layout(s).total);
     const size_t nmask = size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk());
-    const size_t mb = align256(nmask), sb = align256(sla_state_bytes(s));
+    const size_t mb = align256(nmask), sb = align256(sla_state_bytes(s)), ub = align256(sla_sum_bytes(s));
+    const size_t lb = size_t(s.BH()) * size_t(s.N) * kD * sizeof(float);
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(attn + mb + sb + sla_sum_bytes(s), &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, attn + mb + sb + ub + lb, &ws)) != SA_OK) return r;
     uint8_t *keep = ws + attn;
+    float *lin = reinterpret_cast<float *>(ws + attn + mb + sb + ub);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (launch_sla_critical(classes, int64_t(nmask), keep, st) != cudaSuccess) return SA_ERR_CUDA;
-    if ((r = attn_fwd_device(q, k, v, o, s, sm_scale, keep, st)) != SA_OK) return r;
-    return launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws + attn + mb),
-                             reinterpret_cast<float *>(ws + attn + mb + sb), true, o, st) == cudaSuccess
-               ? SA_OK
-               : SA_ERR_CUDA;
+    // the linear part first, in fp32; the sparse part's epilogue adds it to O before O's
+    // only rounding to bf16
+    if (launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws + attn + mb),
+                          reinterpret_cast<float *>(ws + attn + mb + sb), lin, st) != cudaSuccess)
+        return SA_ERR_CUDA;
+    return attn_fwd_device(q, k, v, o, s, sm_scale, keep, st, false, lin);
 }
 
 sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *o, int B, int H, int N, int d,
@@ -640,8 +655,9 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
     if (!block_mask) return attn_fwd_device(q, k, v, o, s, sm_scale, nullptr, st, true);
     // with one: workspace [attention prologue | keep mask intersected with the causal blocks]
     const size_t attn = align256(ws_layout(s).total);
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(attn + size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk()), &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, attn + size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk()), &ws)) != SA_OK) return r;
     if (launch_causal_mask(block_mask, s, ws + attn, st) != cudaSuccess) return SA_ERR_CUDA;
     return attn_fwd_device(q, k, v, o, s, sm_scale, ws + attn, st, true);
 }
@@ -662,8 +678,9 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
         need = std::max(need, align256(ws_layout(s).total));
     }
     if ((r = check_device()) != SA_OK) return r;
+    WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(need, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, need, &ws)) != SA_OK) return r;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // sequence i occupies H * N_i * d consecutive elements of each tensor, after those of
     // the sequences before it; each is an independent [1, H, N_i, d] problem
@@ -758,7 +775,7 @@ sa_status sa_release_workspace(void)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    WsLock lock(g_ws_mutex);
     DeviceWs &w = g_ws[dev];
     if (w.ptr) {
         if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;

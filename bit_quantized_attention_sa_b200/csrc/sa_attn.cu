@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ q_scale,
                     const float *__restrict__ k_scale, const float *__restrict__ v_scale,
                     const uint8_t *__restrict__ mask, __nv_bfloat16 *__restrict__ out, int BH,
-                    int N, int Npad, int nq, int nk, float sm_scale, int causal)
+                    int N, int Npad, int nq, int nk, float sm_scale, int causal,
+                    const float *__restrict__ addend)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -320,10 +321,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = (count_kept(mrow, nk, lane) + 1) / 2;
             const int qrow = qt * 128 + row;
             __nv_bfloat16 *orow = out + (int64_t(bh) * N + qrow) * kD + 64 * wg;
+            // the addend's half row (fp32), added before the one rounding to bf16
+            const float *arow = addend ? addend + (int64_t(bh) * N + qrow) * kD + 64 * wg : nullptr;
             if (n == 0) {
                 if (qrow < N) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < 8; ++c) {
+                        uint32_t w[4] = {0u, 0u, 0u, 0u};
+                        if (arow) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(arow[8 * c + 2 * e], arow[8 * c + 2 * e + 1]);
+                                w[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                        }
+                        reinterpret_cast<uint4 *>(orow)[c] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
                 }
                 continue;
             }
@@ -368,7 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int k = 0; k < 8; ++k) acc[k] = max(acc[k], max(int(a[i + k]), int(b[i + k])));
                     const int imax = max(max(max(acc[0], acc[1]), max(acc[2], acc[3])),
                                          max(max(acc[4], acc[5]), max(acc[6], acc[7])));
-                    pmax = i2f(uint32_t(imax)) * c;
+                    // a block with no key left (ragged tail, causal) gives no maximum,
+                    // whatever its scale
+                    pmax = nvalid > 0 ? i2f(uint32_t(imax)) * c : -INFINITY;
                 }
                 // S has been read: its buffer may take QK of step gg+2
                 tc_fence_before();
@@ -484,8 +499,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 const int i = 8 * cidx + 2 * e;
-                                const float y0 = (__uint_as_float(o[i]) * svp[32 * h + i]) * inv_l;
-                                const float y1 = (__uint_as_float(o[i + 1]) * svp[32 * h + i + 1]) * inv_l;
+                                float y0 = (__uint_as_float(o[i]) * svp[32 * h + i]) * inv_l;
+                                float y1 = (__uint_as_float(o[i + 1]) * svp[32 * h + i + 1]) * inv_l;
+                                if (arow) {
+                                    y0 += arow[32 * h + i];
+                                    y1 += arow[32 * h + i + 1];
+                                }
                                 const __nv_bfloat162 h2 = __floats2bfloat162_rn(y0, y1);
                                 w[e] = *reinterpret_cast<const uint32_t *>(&h2);
                             }
@@ -661,7 +680,7 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st)
     const int grid = ntiles < sms ? ntiles : sms;
     attn_fwd_kernel<<<grid, kThreads, kSmemAlloc, st>>>(a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale,
                                                         a.v_scale, a.mask, a.o, a.BH, a.N, a.Npad,
-                                                        a.nq, a.nk, a.sm_scale, a.causal);
+                                                        a.nq, a.nk, a.sm_scale, a.causal, a.addend);
     return cudaGetLastError();
 }
 

@@ -127,28 +127,83 @@ __device__ __forceinline__ int max64x2(const uint32_t (&a)[32], const uint32_t (
     return max(max(max(acc[0], acc[1]), max(acc[2], acc[3])), max(max(acc[4], acc[5]), max(acc[6], acc[7])));
 }
 
-// 32 keys of S (one array) -> 8 words of e4m3 P = 448 * 2^(S*c2 + nbias); bytes of keys at
-// or past `keep` (index within the array) are zero.
-__device__ __forceinline__ void p_words(const uint32_t (&v)[32], float c2, float nbias, int keep,
-                                        uint32_t (&pw)[8])
+// In-order asm forms of the P steps: their relative order is kept as written.
+__device__ __forceinline__ float cvt_s32_f32_ord(uint32_t x)
 {
+    float y;
+    asm volatile("cvt.rn.f32.s32 %0, %1;" : "=f"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ float fma_ord(float a, float b, float c)
+{
+    float y;
+    asm volatile("fma.rn.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+__device__ __forceinline__ float ex2_ord(float x)
+{
+    float y;
+    asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t pack_e4m3x2_ord(float lo, float hi)
+{
+    uint16_t r;
+    asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// S of one row (128 keys: s0..s3, keys 32a..32a+31 in sa) -> 32 words of e4m3
+// P = 448 * 2^(S*k + nbias), k = k0 for keys 0-63 and k1 for keys 64-127; with MASK, the
+// bytes of keys at or past nv0 (first block) or nv1 (second block) are zero.  The words are
+// computed as a software pipeline -- exponent arguments of word w+1, ex2 of word w, packing
+// of word w-1 -- so that the four ex2 of a word are spread among other instructions: a warp
+// that has the multi-function unit to itself then keeps it busier (10.0 instead of 13.4
+// cycles per 32 keys; the same 8.4 with two warps per scheduler).
+template <bool MASK>
+__device__ __forceinline__ void p_row_impl(const uint32_t (&s0)[32], const uint32_t (&s1)[32],
+                                           const uint32_t (&s2)[32], const uint32_t (&s3)[32],
+                                           float k0, float k1, float nbias, int nv0, int nv1,
+                                           uint32_t (&pw)[32])
+{
+#define SA_SV(key) ((key) < 32 ? s0[(key)] : (key) < 64 ? s1[(key) - 32] : (key) < 96 ? s2[(key) - 64] : s3[(key) - 96])
+    float y[2][4], e[2][4];
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-        float y0, y1, y2, y3;
-        fma2(y0, y1, i2f(v[4 * w]), i2f(v[4 * w + 1]), c2, c2, nbias, nbias);
-        fma2(y2, y3, i2f(v[4 * w + 2]), i2f(v[4 * w + 3]), c2, c2, nbias, nbias);
-        const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
-        const float e2 = SA_POLY_OF_4 >= 2 ? exp2_poly(y2) : ex2_approx(y2);
-        const float e3 = SA_POLY_OF_4 >= 1 ? exp2_poly(y3) : ex2_approx(y3);
-        pw[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
-    }
-    if (keep < 32) {
+    for (int i = 0; i < 4; ++i) y[0][i] = fma_ord(cvt_s32_f32_ord(SA_SV(i)), k0, nbias);
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const int kb = keep - 4 * w;  // bytes of this word to keep
-            pw[w] = kb >= 4 ? pw[w] : (kb <= 0 ? 0u : (pw[w] & ((1u << (8 * kb)) - 1u)));
+    for (int w = 0; w < 33; ++w) {
+        const int cur = w & 1, nxt = cur ^ 1;
+        if (w + 1 < 32) {
+            const float k = (w + 1) < 16 ? k0 : k1;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[nxt][i] = fma_ord(cvt_s32_f32_ord(SA_SV(4 * (w + 1) + i)), k, nbias);
+        }
+        if (w < 32) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) e[cur][i] = ex2_ord(y[cur][i]);
+        }
+        if (w >= 1) {
+            uint32_t x = pack_e4m3x2_ord(e[nxt][0], e[nxt][1]) | (pack_e4m3x2_ord(e[nxt][2], e[nxt][3]) << 16);
+            if (MASK) {
+                const int kb = ((w - 1) < 16 ? nv0 : nv1) - 4 * ((w - 1) & 15);  // bytes to keep
+                x = kb >= 4 ? x : (kb <= 0 ? 0u : (x & ((1u << (8 * kb)) - 1u)));
+            }
+            pw[w - 1] = x;
         }
     }
+#undef SA_SV
+}
+
+// The masked form only where some row of the warp has a partial block (ragged tail, causal).
+__device__ __forceinline__ void p_row(const uint32_t (&s0)[32], const uint32_t (&s1)[32],
+                                      const uint32_t (&s2)[32], const uint32_t (&s3)[32],
+                                      float k0, float k1, float nbias, int nv0, int nv1,
+                                      uint32_t (&pw)[32])
+{
+    if (__any_sync(0xffffffffu, nv0 < 64 || nv1 < 64))
+        p_row_impl<true>(s0, s1, s2, s3, k0, k1, nbias, nv0, nv1, pw);
+    else
+        p_row_impl<false>(s0, s1, s2, s3, k0, k1, nbias, nv0, nv1, pw);
 }
 
 }  // namespace pairs
@@ -190,7 +245,7 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
     using pairs::setmaxnreg_dec;
     using pairs::tmem_ld128;
     using pairs::max64x2;
-    using pairs::p_words;
+    using pairs::p_row;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
@@ -386,8 +441,9 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                     tmem_ld128(sa, s0, s1, s2, s3);
                 }
 
-                // keys past the end of the sequence (last block only) drop out of the max
-                // (their P bytes are cleared below)
+                // keys past the end of the sequence or after the row (causal) drop out of
+                // the max (their P bytes are cleared below); a block with no key left
+                // contributes no maximum at all, whatever its scale
                 if (nv0 < 64) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -402,10 +458,10 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                         if (i + 32 >= nv1) s3[i] = uint32_t(INT_MIN);
                     }
                 }
-                // row max on int32 S per block (each scale is positive, so max commutes)
+                // row max on int32 S per block (each scale is non-negative, so max commutes)
                 const float c0 = (sq * ks0) * sm_scale, c1 = (sq * ks1) * sm_scale;
-                float pmax = i2f(uint32_t(max64x2(s0, s1))) * c0;
-                if (two) pmax = fmaxf(pmax, i2f(uint32_t(max64x2(s2, s3))) * c1);
+                float pmax = nv0 > 0 ? i2f(uint32_t(max64x2(s0, s1))) * c0 : -INFINITY;
+                if (nv1 > 0) pmax = fmaxf(pmax, i2f(uint32_t(max64x2(s2, s3))) * c1);
                 const float mnew = fmaxf(m, pmax);
                 // the S buffer goes to the other tile's QK only now, after the maximum: this
                 // delays the other warpgroup by about that long, so that its exponentials
@@ -418,17 +474,8 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
 
                 // P = e4m3(448 * 2^(S*c*log2e - mnew*log2e)), 8 words per 32 keys
                 const float nbias = kLog2_448 - mnew * kLog2e;
-                uint32_t pw[4][8];
-                p_words(s0, c0 * kLog2e, nbias, nv0, pw[0]);
-                p_words(s1, c0 * kLog2e, nbias, nv0 - 32, pw[1]);
-
-                if (two) {
-                    p_words(s2, c1 * kLog2e, nbias, nv1, pw[2]);
-                    p_words(s3, c1 * kLog2e, nbias, nv1 - 32, pw[3]);
-                } else {
-#pragma unroll
-                    for (int w = 0; w < 8; ++w) pw[2][w] = pw[3][w] = 0u;
-                }
+                uint32_t pw[32];
+                p_row(s0, s1, s2, s3, c0 * kLog2e, c1 * kLog2e, nbias, nv0, two ? nv1 : 0, pw);
 
                 // the P tile and O are free once the PV of the previous step completed
                 if (c >= 1 && ok) ok = mbar_wait(bar(kBarPvDone + t), (c - 1) & 1, abort_flag);
@@ -437,8 +484,7 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     *reinterpret_cast<uint4 *>(prow + ((k ^ (row & 7)) << 4)) =
-                        make_uint4(pw[k >> 1][4 * (k & 1)], pw[k >> 1][4 * (k & 1) + 1],
-                                   pw[k >> 1][4 * (k & 1) + 2], pw[k >> 1][4 * (k & 1) + 3]);
+                        make_uint4(pw[4 * k], pw[4 * k + 1], pw[4 * k + 2], pw[4 * k + 3]);
 
                 // rescale O (and its row-sum column) when the running max grew
                 if (j > 0) {

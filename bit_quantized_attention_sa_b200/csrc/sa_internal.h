@@ -48,6 +48,8 @@ struct AttnArgs {
     int BH, N, Npad, nq, nk;
     float sm_scale;
     int causal = 0;  // row r keeps only the keys t <= r (mask must then be set)
+    // fp32 [B,H,N,d] added to O before its single rounding to bf16 (masked calls), or null
+    const float *addend = nullptr;
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
 cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k, int BH,
@@ -77,11 +79,10 @@ cudaError_t read_and_clear_w8a8_status(int *status);
 // ---- SLA linear branch (sa_sla.cu)
 size_t sla_state_bytes(const Shape &s);  // per-key-block states, fp32
 size_t sla_sum_bytes(const Shape &s);    // per-query-block summed states, fp32
-// The branch for all rows: fp32 out [B,H,N,d] (add_into_bf16 false) or added to the bf16
-// out (true).  classes uint8 [B,H,nq,nk] (1 = marginal); proj fp32 [d][d] or null.
+// The branch for all rows: fp32 out [B,H,N,d].  classes uint8 [B,H,nq,nk] (1 = marginal);
+// proj fp32 [d][d] or null.
 cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, const Shape &s,
-                              int phi, const float *proj, float *state, float *sums, bool add_into_bf16, void *out,
-                              cudaStream_t st);
+                              int phi, const float *proj, float *state, float *sums, float *out, cudaStream_t st);
 // keep[e] = classes[e] >= 2 (the sparse part's block mask), n entries.
 cudaError_t launch_sla_critical(const uint8_t *classes, int64_t n, uint8_t *keep, cudaStream_t st);
 // Reads and clears the device status word of the current device (synchronous).

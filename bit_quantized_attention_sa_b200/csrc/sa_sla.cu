@@ -194,12 +194,10 @@ constexpr int kApplyPhi = 0, kApplyState = kD * kApplyLd, kApplyDen = kApplyStat
 constexpr int kApplySmemFloats = kApplyDen + kD;
 constexpr size_t kApplySmemBytes = size_t(kApplySmemFloats) * sizeof(float);
 
-// grid (nq, BH), 256 threads.  out: fp32 [BH, N, d] (ADD false) or the bf16 output the
-// branch is added to (ADD true).  proj: fp32 [d][d] or null (identity).
-template <bool ADD>
+// grid (nq, BH), 256 threads.  out: fp32 [BH, N, d].  proj: fp32 [d][d] or null (identity).
 __global__ void __launch_bounds__(256)
     sla_apply_kernel(const uint16_t *__restrict__ q, const float *__restrict__ sums, const float *__restrict__ proj,
-                     int N, int nq, int phi, void *__restrict__ out)
+                     int N, int nq, int phi, float *__restrict__ out)
 {
     extern __shared__ __align__(16) float sm[];
     float *pq = sm + kApplyPhi, *st = sm + kApplyState, *den = sm + kApplyDen;
@@ -296,25 +294,9 @@ __global__ void __launch_bounds__(256)
     for (int m = 0; m < 8; ++m) {
         const int64_t tok = int64_t(i) * kQBlk + ty + 16 * m;
         if (tok >= N) continue;
-        const int64_t off = (bh * N + tok) * kD + 8 * tx;
-        if (ADD) {
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out) + off;
-            const uint4 old = *reinterpret_cast<const uint4 *>(o);
-            const uint32_t w[4] = {old.x, old.y, old.z, old.w};
-            uint32_t nw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float lo = __uint_as_float(w[e] << 16) + acc[m][2 * e];
-                const float hi = __uint_as_float(w[e] & 0xFFFF0000u) + acc[m][2 * e + 1];
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
-                nw[e] = *reinterpret_cast<const uint32_t *>(&h2);
-            }
-            *reinterpret_cast<uint4 *>(o) = make_uint4(nw[0], nw[1], nw[2], nw[3]);
-        } else {
-            float *o = static_cast<float *>(out) + off;
-            *reinterpret_cast<float4 *>(o) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-            *reinterpret_cast<float4 *>(o + 4) = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
-        }
+        float *o = out + (bh * N + tok) * kD + 8 * tx;
+        *reinterpret_cast<float4 *>(o) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+        *reinterpret_cast<float4 *>(o + 4) = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
     }
 }
 
@@ -330,8 +312,7 @@ size_t sla_state_bytes(const Shape &s) { return size_t(s.BH()) * size_t(s.nk()) 
 size_t sla_sum_bytes(const Shape &s) { return size_t(s.BH()) * size_t(s.nq()) * kStateFloats * sizeof(float); }
 
 cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, const Shape &s,
-                              int phi, const float *proj, float *state, float *sums, bool add_into_bf16, void *out,
-                              cudaStream_t st)
+                              int phi, const float *proj, float *state, float *sums, float *out, cudaStream_t st)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -343,9 +324,7 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
                                       int(state_smem))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_state_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(sizeof(uint32_t) * kMaskMaxKeyBlocks))) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(sla_apply_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(kApplySmemBytes))) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(sla_apply_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            (e = cudaFuncSetAttribute(sla_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(kApplySmemBytes))) != cudaSuccess)
             return e;
         attr_set[dev] = true;
@@ -359,10 +338,7 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
                            256, sizeof(uint32_t) * size_t(nk), st>>>(state, classes, nq, nk, sums);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const dim3 ga(unsigned(nq), unsigned(s.BH()));
-    if (add_into_bf16)
-        sla_apply_kernel<true><<<ga, 256, kApplySmemBytes, st>>>(qb, sums, proj, N, nq, phi, out);
-    else
-        sla_apply_kernel<false><<<ga, 256, kApplySmemBytes, st>>>(qb, sums, proj, N, nq, phi, out);
+    sla_apply_kernel<<<ga, 256, kApplySmemBytes, st>>>(qb, sums, proj, N, nq, phi, out);
     return cudaGetLastError();
 }
 

@@ -42,6 +42,20 @@
  *     expire set a device status word read by sa_get_device_status.
  *   - Block mask: uint8 [B,H,nq,nk], nonzero keeps the (128-query x 64-key) block; NULL
  *     keeps every block.  Masked blocks are neither loaded nor computed.
+ *   - Library workspace.  The entry points marked "uses the library workspace" keep their
+ *     intermediates (quantised Q/K/V, scales, partial sums, masks, SLA states) in ONE
+ *     buffer per device, owned by the library and grown on demand.  Growing it
+ *     synchronises the device and frees the old buffer; the library holds a lock from a
+ *     call's workspace request until that call's launches are enqueued, so calls from
+ *     several host threads cannot free memory another call is about to use.  The buffer
+ *     is NOT per stream: two such calls in flight at once on different streams of one
+ *     device overwrite each other's intermediates and give wrong results without any
+ *     error.  Order such calls on one stream (or with events).  sa_attn_fwd_quantized,
+ *     sa_debug_qk_s32 and sa_w8a8_gemm use no workspace; sa_quantize_qk_noalloc uses its
+ *     own fixed array (see there).
+ *   - The library caches per-device state (the workspace, tensor-map encoder, kernel
+ *     attributes and the scratch array's address) for the life of the process: do not use
+ *     it across cudaDeviceReset.
  */
 #ifndef SA_H
 #define SA_H
@@ -231,7 +245,9 @@ sa_status sa_sla_linear(const void *q, const void *k, const void *v, const uint8
 
 /* The SLA forward: o bf16 [B,H,N,d] = the quantised attention of sa_attn_fwd restricted to
  * the critical blocks (a row without one gives 0), plus the projected linear branch,
- * added in fp32 and rounded once to bf16. */
+ * added in fp32 and rounded once to bf16.  The linear branch runs first, into the library
+ * workspace in fp32 (a further 4 * d bytes per query token), and the sparse part's
+ * epilogue adds it to O before O's only rounding. */
 sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B, int H, int N, int d,
                      float sm_scale, const uint8_t *classes, int phi, const float *proj, void *stream);
 
