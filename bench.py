@@ -155,29 +155,60 @@ class ClockSampler:
 # ------------------------------------------------------------------------ CPU oracle arm
 
 
-def oracle_sample(w, q, k, v, m, rows_per_head: int):
-    """Times the CPU oracle on a bounded sample of the workload: the prologue of one head
-    and `rows_per_head` query rows of it.  Returns (ops_equiv, seconds, description)."""
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, q, k, v, m, threads: int, heads: int, rows_per_block=None):
+    """Times the CPU oracle, as it stands, on a bounded sample of the workload: for each of
+    the first `heads` heads its prologue (K mean, Q/K and V quantisation) and the query rows
+    of its first and its ragged last 128-query block (the first `rows_per_block` rows of
+    each, if given).  `threads` host threads run disjoint (head, block) units; each calls the
+    single-threaded C oracle, which releases the interpreter lock.  The prologue of a head
+    serves all N of its rows, so the sampled rows are charged their share of its time.
+    Returns (ops_equivalent, seconds, description, threads)."""
+    import concurrent.futures as cf
     import oracle
     oracle.build()
-    h = 0
-    qh, kh, vh = (np.ascontiguousarray(x[:1, h:h + 1]) for x in (q, k, v))
-    mh = np.ascontiguousarray(m[:1, h:h + 1]) if m is not None else None
-    t0 = time.perf_counter()
-    qk = oracle.quantize_qk(qh, kh)
-    vq = oracle.quantize_v(vh)
-    t_pro = time.perf_counter() - t0
-    rng = np.random.default_rng(0)
-    rows = [(0, int(r)) for r in rng.choice(w.N, size=rows_per_head, replace=False)]
-    t0 = time.perf_counter()
-    oracle.attn_rows(qk, vq, w.N, w.sm_scale, rows, mh, 2)
-    t_rows = time.perf_counter() - t0
-    # the prologue serves all N rows of the head: charge the sampled rows their share
-    secs = t_rows + t_pro * rows_per_head / w.N
-    ops = 4.0 * rows_per_head * w.N * w.d
-    desc = (f"1 head of {w.name}: prologue ({t_pro:.2f} s, charged {rows_per_head}/{w.N}) + "
-            f"{rows_per_head} random query rows ({t_rows:.2f} s); single-threaded C oracle")
-    return ops, secs, desc
+    nq = -(-w.N // 128)
+    blocks = [0] if nq == 1 else [0, nq - 1]
+    heads = max(1, min(heads, w.B * w.H))
+    hsel = [(b, h) for b in range(w.B) for h in range(w.H)][:heads]
+
+    def prologue(bh):
+        b, h = bh
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        qh, kh, vh = (np.ascontiguousarray(x[sl]) for x in (q, k, v))
+        mh = np.ascontiguousarray(m[sl]) if m is not None else None
+        return oracle.quantize_qk(qh, kh), oracle.quantize_v(vh), mh
+
+    def rows_of(blk):
+        lo, hi = 128 * blk, min(128 * blk + 128, w.N)
+        if rows_per_block is not None:
+            hi = min(hi, lo + rows_per_block)
+        return [(0, r) for r in range(lo, hi)]
+
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        t0 = time.perf_counter()
+        pro = list(ex.map(prologue, hsel))
+        t_pro = time.perf_counter() - t0
+        units = [(i, blk) for i in range(len(hsel)) for blk in blocks]
+        t0 = time.perf_counter()
+        list(ex.map(lambda u: oracle.attn_rows(pro[u[0]][0], pro[u[0]][1], w.N, w.sm_scale, rows_of(u[1]),
+                                               pro[u[0]][2], 2), units))
+        t_rows = time.perf_counter() - t0
+    nrows = sum(len(rows_of(blk)) for blk in blocks)  # per head
+    secs = t_rows + t_pro * nrows / w.N
+    ops = 4.0 * nrows * len(hsel) * w.N * w.d
+    what = "all rows" if rows_per_block is None else f"the first {rows_per_block} rows"
+    desc = (f"{len(hsel)} head(s) of {w.name}: {what} of the first and ragged last query blocks "
+            f"({nrows} rows per head, {t_rows:.2f} s) + their prologues ({t_pro:.2f} s, charged {nrows}/{w.N}); "
+            f"C oracle, {threads} host thread(s) over {len(units)} (head, block) units; rate extrapolated to "
+            f"the whole workload")
+    return ops, secs, desc, threads
 
 
 def run_reference(args, w):
@@ -185,11 +216,12 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     q, k, v, m = make_workload(w)
-    rows = args.oracle_rows
+    cores = host_cores()
+    heads = max(1, cores // 2)
     vals = []
     desc = ""
     for i in range(args.warmup + args.steps):
-        ops, secs, desc = oracle_sample(w, q, k, v, m, rows)
+        ops, secs, desc, _ = oracle_sample(w, q, k, v, m, cores, heads, args.oracle_rows)
         if i >= args.warmup:
             vals.append(ops / secs / 1e12)
     value = float(np.median(vals)) if vals else 0.0
@@ -202,8 +234,8 @@ def run_reference(args, w):
         "dtype": "int8+fp8e4m3 (emulated in fp32 on the CPU)", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "mask_density": w.mask_density, "sample": desc},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc, "extrapolated": True},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -221,8 +253,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--oracle-rows", type=int, default=64,
-                    help="query rows in the CPU oracle sample")
+    ap.add_argument("--oracle-rows", type=int, default=16,
+                    help="rows per query block in each step of the reference arm's oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sla", action="store_true", help="skip the SLA forward timing")
     ap.add_argument("--no-causal", action="store_true", help="skip the causal forward timing")
@@ -305,7 +337,50 @@ def main():
     a1.record(stream)
     barrier()
     t_attn = slowest(a0.elapsed_time(a1) / 1e3 / args.steps)
+
+    # ---- the prologue alone (K mean, Q/K INT8, V FP8 into caller buffers): reported on its
+    # own, as the selector/pack/dequant cost of a low-bit attention step
+    for _ in range(args.warmup):
+        sa.sa_quantize_qk(dq, dk)
+        sa.sa_quantize_v(dv)
+    barrier()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(args.steps):
+        sa.sa_quantize_qk(dq, dk)
+        sa.sa_quantize_v(dv)
+    g1.record(stream)
+    barrier()
+    t_pro = slowest(g0.elapsed_time(g1) / 1e3 / args.steps)
+    # bytes per (token, channel): read K (mean), Q and K (codes), V twice (maximum, codes) in bf16;
+    # write q8, k8, v8: 2 + 4 + 4 + 3 = 13
+    pro_bytes = 13 * w.B * w.H * w.N * w.d
+    prologue = {"ms": t_pro * 1e3, "share_of_step": t_pro / t_step,
+                "steps": "sa_quantize_qk (K mean, Q INT8, smoothed K INT8) + sa_quantize_v (V FP8, transposed)",
+                "algorithmic_bytes": pro_bytes, "gbs": pro_bytes / t_pro / 1e9}
     del q8, k8, vt
+
+    # ---- this device's own 8-bit tensor-core rate: chains of four M128 N256 K32 tcgen05
+    # MMAs from every SM, kind::i8 and kind::f8f6f4 (e4m3), timed on the stream
+    def mma_rate(kind):
+        sa.sa_debug_mma_peak(kind, 256)
+        best = 0.0
+        for _ in range(5):
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0.record(stream)
+            ops_p = sa.sa_debug_mma_peak(kind, 65536)
+            r1.record(stream)
+            torch.cuda.synchronize(dev)
+            best = max(best, ops_p / (r0.elapsed_time(r1) * 1e-3) / 1e12)
+        return best
+    peak_sampler = ClockSampler(local_rank)
+    peak_sampler.start()
+    time.sleep(0.2)
+    peak_i8, peak_f8 = mma_rate(0), mma_rate(1)
+    peak_clocks = peak_sampler.stop()
+    assert sa.sa_get_device_status() == 0
+    # the attention kernel's operations are half kind::i8 (Q.K^T) and half e4m3 (P.V)
+    peak_8bit = 2.0 / (1.0 / peak_i8 + 1.0 / peak_f8)
 
     # ---- end to end through the public API with host buffers: sa_attn_fwd_host uploads
     # q, k, v (and the mask) from page-locked memory and downloads O, in chunks of heads
@@ -365,8 +440,8 @@ def main():
         barrier()
         t_causal = slowest(c0.elapsed_time(c1) / 1e3 / args.steps)
         assert sa.sa_get_device_status() == 0
-        causal = {"step": "sa_attn_fwd_causal: prologue + masked kernel over the blocks up to the diagonal, "
-                          "keys after each row dropped",
+        causal = {"step": "sa_attn_fwd_causal: prologue + the two-tile kernel over the blocks up to each "
+                          "tile pair's diagonal, keys after each row dropped",
                   "ms": t_causal * 1e3, "executed_block_fraction": blocks / (w.B * w.H * nq * nk),
                   "executed_tops": whole_job_tops(ops_causal, world, t_causal)}
 
@@ -450,9 +525,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ops_c, secs_c, desc = oracle_sample(w, q, k, v, m, args.oracle_rows)
-        cpu = {"value": ops_c / secs_c / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-               "sample": desc}
+        # two legs of the oracle as it stands, on the host cores of this run: one thread on one
+        # head, and one thread per host core over heads x (first, last) query blocks
+        cores = host_cores()
+        ops1, secs1, desc1, _ = oracle_sample(w, q, k, v, m, 1, 1)
+        opsn, secsn, descn, _ = oracle_sample(w, q, k, v, m, cores, max(1, cores // 2))
+        cpu = {"value": opsn / secsn / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": descn, "extrapolated": True,
+               "single_threaded": {"value": ops1 / secs1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                   "sample": desc1, "extrapolated": True}}
 
     if rank == 0:
         line = {
@@ -469,6 +550,12 @@ def main():
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "peak_source": peak_src,
                          "frac_of_datasheet_4500": achieved / DATASHEET_TOPS,
+                         "measured_8bit_mma": {"i8_tops": peak_i8, "e4m3_tops": peak_f8, "combined_tops": peak_8bit,
+                                               "frac": achieved / peak_8bit, "clocks": peak_clocks,
+                                               "how": "sa_debug_mma_peak: every SM issues chains of four "
+                                                      "M128 N256 K32 tcgen05 MMAs from shared memory, CUDA "
+                                                      "events, best of 5; combined = harmonic mean (the "
+                                                      "kernel's ops are half of each kind)"},
                          "ms_per_launch": t_attn * 1e3,
                          "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
             "cpu_baseline": cpu,
@@ -477,6 +564,7 @@ def main():
                     "ms_per_step": t_e2e * 1e3},
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clocks,
+            "prologue": prologue,
         }
         if causal is not None:
             line["causal"] = causal

@@ -42,7 +42,7 @@ _lib.sa_w8a8_linear.argtypes = [_P, _P, _P, _I, _I, _I, _P, _P]
 _lib.sa_sla_linear.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]
 _lib.sa_sla_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _I, _P, _P]
 _lib.sa_debug_wait_timeout.argtypes = [_I, _P]
-_lib.sa_debug_exp2_poly.argtypes = [_P, _P, _I, _P]
+_lib.sa_debug_mma_peak.argtypes = [_I, _I, _P]
 _lib.sa_get_device_status.argtypes = []
 _lib.sa_status_string.argtypes = [_I]
 _lib.sa_status_string.restype = ctypes.c_char_p
@@ -54,7 +54,7 @@ _lib.sa_padded_len.restype = ctypes.c_int64
 for _name in ("sa_quantize_qk", "sa_quantize_qk_noalloc", "sa_quantize_v", "sa_attn_fwd", "sa_attn_fwd_host",
               "sa_attn_fwd_causal", "sa_attn_fwd_varlen",
               "sa_attn_fwd_quantized",
-              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_sla_linear", "sa_sla_fwd", "sa_debug_wait_timeout", "sa_debug_exp2_poly", "sa_get_device_status",
+              "sa_debug_qk_s32", "sa_block_mask", "sa_debug_pool", "sa_w8a8_quantize", "sa_w8a8_gemm", "sa_w8a8_linear", "sa_sla_linear", "sa_sla_fwd", "sa_debug_wait_timeout", "sa_debug_mma_peak", "sa_get_device_status",
               "sa_release_workspace"):
     getattr(_lib, _name).restype = _I
 
@@ -405,13 +405,13 @@ def sa_debug_wait_timeout(timeout_us: int, device=None):
     _check(_lib.sa_debug_wait_timeout(int(timeout_us), _stream(dev)), "sa_debug_wait_timeout")
 
 
-def sa_debug_exp2_poly(x: torch.Tensor) -> torch.Tensor:
-    """2^x by the attention kernel's polynomial exponential (fp32 CUDA tensor)."""
-    _need(x, torch.float32, "x")
-    y = torch.empty_like(x)
-    _check(_lib.sa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(x.device)),
-           "sa_debug_exp2_poly")
-    return y
+def sa_debug_mma_peak(kind: int, reps: int, device=None):
+    """Launches the tensor-core rate kernel on the current stream (kind 0: kind::i8, 1: e4m3
+    kind::f8f6f4); the caller times it.  Returns the operations it performs."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _check(_lib.sa_debug_mma_peak(kind, reps, _stream(dev)), "sa_debug_mma_peak")
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return float(sms) * reps * 4 * 2 * 128 * 256 * 32
 
 
 def sa_get_device_status() -> int:

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsa.so")
-SOURCES = ["sa_api.cu", "sa_prologue.cu", "sa_attn.cu", "sa_mask.cu", "sa_w8a8.cu", "sa_sla.cu"]
+SOURCES = ["sa_api.cu", "sa_prologue.cu", "sa_attn.cu", "sa_mask.cu", "sa_w8a8.cu", "sa_sla.cu", "sa_peak.cu"]
 HEADERS = ["sa_ptx.cuh", "sa_internal.h", "sa_attn_pairs.cuh"]
 
 NVCC_FLAGS = [

@@ -728,23 +728,21 @@ sa_status sa_debug_wait_timeout(int timeout_us, void *stream)
                : SA_ERR_CUDA;
 }
 
-sa_status sa_debug_exp2_poly(const float *x, float *y, int n, void *stream)
+sa_status sa_debug_mma_peak(int kind, int reps, void *stream)
 {
-    if (n < 1) return SA_ERR_INVALID_ARG;
-    sa_status r = check_ptrs({x, y});
+    if ((kind != 0 && kind != 1) || reps < 1 || reps > (1 << 20)) return SA_ERR_INVALID_ARG;
+    sa_status r = check_device();
     if (r != SA_OK) return r;
-    if ((r = check_device()) != SA_OK) return r;
-    return launch_debug_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? SA_OK
-               : SA_ERR_CUDA;
+    return launch_mma_peak(kind, reps, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 sa_status sa_get_device_status(void)
 {
-    int st = 0, st_w8a8 = 0;
-    if (read_and_clear_status(&st) != cudaSuccess || read_and_clear_w8a8_status(&st_w8a8) != cudaSuccess)
+    int st = 0, st_w8a8 = 0, st_peak = 0;
+    if (read_and_clear_status(&st) != cudaSuccess || read_and_clear_w8a8_status(&st_w8a8) != cudaSuccess ||
+        read_and_clear_peak_status(&st_peak) != cudaSuccess)
         return SA_ERR_CUDA;
-    return st == 0 && st_w8a8 == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
+    return st == 0 && st_w8a8 == 0 && st_peak == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
 }
 
 const char *sa_status_string(sa_status s)

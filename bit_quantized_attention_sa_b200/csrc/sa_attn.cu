@@ -83,12 +83,6 @@ static_assert(kVHalfBytes % 1024 == 0, "V half tiles stay 1024-B aligned");
 constexpr uint32_t kIdescQK = idesc_s8_s32(128, 128);
 constexpr uint32_t kIdescPV = idesc_e4m3_f32(128, kOCols);
 
-// Of every 4 softmax exponentials, this many run as a polynomial on the FMA/ALU pipes
-// (exp2_poly) instead of the MUFU pipe, to balance the two.
-#ifndef SA_POLY_OF_4
-#define SA_POLY_OF_4 0
-#endif
-
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;
 
@@ -111,6 +105,68 @@ __device__ __forceinline__ int count_kept(const uint8_t *mrow, int nk, int lane)
 }
 
 __device__ __forceinline__ float i2f(uint32_t x) { return __int2float_rn(int(x)); }
+
+// In-order asm forms of the P steps: their relative order is kept as written.
+__device__ __forceinline__ float cvt_s32_f32_ord(uint32_t x)
+{
+    float y;
+    asm volatile("cvt.rn.f32.s32 %0, %1;" : "=f"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ float fma_ord(float a, float b, float c)
+{
+    float y;
+    asm volatile("fma.rn.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+__device__ __forceinline__ float ex2_ord(float x)
+{
+    float y;
+    asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t pack_e4m3x2_ord(float lo, float hi)
+{
+    uint16_t r;
+    asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// 64 keys of S (a: keys 0-31, b: keys 32-63) -> 16 words of e4m3 P = 448 * 2^(S*k +
+// nbias); with MASK, bytes of keys at or past nvalid are zero.  Computed as a software
+// pipeline (exponent arguments of word w+1, ex2 of word w, packing of word w-1), as the
+// 128-key row of the pair kernel, so that a warp alone in this phase keeps the
+// multi-function unit busier.
+template <bool MASK>
+__device__ __forceinline__ void p_half_impl(const uint32_t (&a)[32], const uint32_t (&b)[32], float k,
+                                            float nbias, int nvalid, uint32_t (&pw)[16])
+{
+#define SA_HV(key) ((key) < 32 ? a[(key)] : b[(key) - 32])
+    float y[2][4], e[2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) y[0][i] = fma_ord(cvt_s32_f32_ord(SA_HV(i)), k, nbias);
+#pragma unroll
+    for (int w = 0; w < 17; ++w) {
+        const int cur = w & 1, nxt = cur ^ 1;
+        if (w + 1 < 16) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[nxt][i] = fma_ord(cvt_s32_f32_ord(SA_HV(4 * (w + 1) + i)), k, nbias);
+        }
+        if (w < 16) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) e[cur][i] = ex2_ord(y[cur][i]);
+        }
+        if (w >= 1) {
+            uint32_t x = pack_e4m3x2_ord(e[nxt][0], e[nxt][1]) | (pack_e4m3x2_ord(e[nxt][2], e[nxt][3]) << 16);
+            if (MASK) {
+                const int kb = nvalid - 4 * (w - 1);  // bytes of this word to keep
+                x = kb >= 4 ? x : (kb <= 0 ? 0u : (x & ((1u << (8 * kb)) - 1u)));
+            }
+            pw[w - 1] = x;
+        }
+    }
+#undef SA_HV
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -401,25 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (j >= 0) {
                     const float c2 = c * kLog2e;
                     const float nb = kLog2_448 - mnew * kLog2e;
-#pragma unroll
-                    for (int w = 0; w < 16; ++w) {
-                        const uint32_t *src = w < 8 ? a : b;
-                        const int i = 4 * (w & 7);
-                        float y0, y1, y2, y3;
-                        fma2(y0, y1, i2f(src[i]), i2f(src[i + 1]), c2, c2, nb, nb);
-                        fma2(y2, y3, i2f(src[i + 2]), i2f(src[i + 3]), c2, c2, nb, nb);
-                        const float e0 = ex2_approx(y0), e1 = ex2_approx(y1);
-                        const float e2 = SA_POLY_OF_4 >= 2 ? exp2_poly(y2) : ex2_approx(y2);
-                        const float e3 = SA_POLY_OF_4 >= 1 ? exp2_poly(y3) : ex2_approx(y3);
-                        pw[w] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
-                    }
-                    if (nvalid < 64) {
-#pragma unroll
-                        for (int w = 0; w < 16; ++w) {
-                            const int keep = nvalid - 4 * w;  // bytes of this word to keep
-                            pw[w] = keep >= 4 ? pw[w] : (keep <= 0 ? 0u : (pw[w] & ((1u << (8 * keep)) - 1u)));
-                        }
-                    }
+                    // the masked form only where some row of the warp has a partial block
+                    if (__any_sync(0xffffffffu, nvalid < 64))
+                        p_half_impl<true>(a, b, c2, nb, nvalid, pw);
+                    else
+                        p_half_impl<false>(a, b, c2, nb, nvalid, pw);
                 } else {
 #pragma unroll
                     for (int w = 0; w < 16; ++w) pw[w] = 0u;
@@ -617,23 +659,9 @@ __global__ void debug_wait_timeout_kernel(unsigned long long timeout_ns)
     }
 }
 
-// Debug: the softmax's polynomial exp2 applied elementwise, for checking it against the
-// CUDA math library.
-__global__ void debug_exp2_poly_kernel(const float *__restrict__ x, float *__restrict__ y, int n)
-{
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) y[i] = exp2_poly(x[i]);
-}
-
 #include "sa_attn_pairs.cuh"
 
 }  // namespace
-
-cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t st)
-{
-    debug_exp2_poly_kernel<<<(n + 255) / 256, 256, 0, st>>>(x, y, n);
-    return cudaGetLastError();
-}
 
 // Without a mask: two query tiles per CTA (attn_pairs_kernel).
 static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)

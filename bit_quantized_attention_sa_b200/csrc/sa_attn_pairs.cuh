@@ -127,32 +127,6 @@ __device__ __forceinline__ int max64x2(const uint32_t (&a)[32], const uint32_t (
     return max(max(max(acc[0], acc[1]), max(acc[2], acc[3])), max(max(acc[4], acc[5]), max(acc[6], acc[7])));
 }
 
-// In-order asm forms of the P steps: their relative order is kept as written.
-__device__ __forceinline__ float cvt_s32_f32_ord(uint32_t x)
-{
-    float y;
-    asm volatile("cvt.rn.f32.s32 %0, %1;" : "=f"(y) : "r"(x));
-    return y;
-}
-__device__ __forceinline__ float fma_ord(float a, float b, float c)
-{
-    float y;
-    asm volatile("fma.rn.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
-    return y;
-}
-__device__ __forceinline__ float ex2_ord(float x)
-{
-    float y;
-    asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ uint32_t pack_e4m3x2_ord(float lo, float hi)
-{
-    uint16_t r;
-    asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
 // S of one row (128 keys: s0..s3, keys 32a..32a+31 in sa) -> 32 words of e4m3
 // P = 448 * 2^(S*k + nbias), k = k0 for keys 0-63 and k1 for keys 64-127; with MASK, the
 // bytes of keys at or past nv0 (first block) or nv1 (second block) are zero.  The words are

@@ -55,7 +55,6 @@ cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
 cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k, int BH,
                                 int Npad, int32_t *s_out, cudaStream_t st);
 cudaError_t launch_debug_wait_timeout(int timeout_us, cudaStream_t st);
-cudaError_t launch_debug_exp2_poly(const float *x, float *y, int n, cudaStream_t st);
 // ---- block-mask producer (sa_mask.cu)
 constexpr int kMaskMaxKeyBlocks = 4096;  // key blocks per mask row the selector sorts in shared memory
 cudaError_t launch_pool_qk(const void *q, const void *k, const Shape &s, float *qbar, float *kbar,
@@ -87,6 +86,10 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
 cudaError_t launch_sla_critical(const uint8_t *classes, int64_t n, uint8_t *keep, cudaStream_t st);
 // Reads and clears the device status word of the current device (synchronous).
 cudaError_t read_and_clear_status(int *status);
+// ---- measured tensor-core peak (sa_peak.cu): one CTA per SM, reps chains of four
+// M128 N256 K32 MMAs (kind 0: i8, kind 1: e4m3), 2*128*256*32 operations per MMA
+cudaError_t launch_mma_peak(int kind, int reps, cudaStream_t st);
+cudaError_t read_and_clear_peak_status(int *status);
 
 // ---- tensor maps (sa_api.cu)
 bool encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,

@@ -356,41 +356,6 @@ __device__ __forceinline__ void mul2(float &d0, float &d1, float a0, float a1, f
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 2^x on the FMA/ALU pipes, for x <= 9 (results feed an e4m3 cast, which keeps 3 mantissa
-// bits).  Cody-Waite range reduction x = n + f with n = round(x), |f| <= 1/2, then a cubic
-// fitted to 2^f on [-1/2, 1/2] by iterated weighted least squares for minimum relative
-// error (max relative error 7.5e-5 in fp32 Horner form), then n added to the exponent
-// field.  x is clamped at -16: 2^-16 is below half the smallest e4m3 subnormal (2^-9), so
-// every clamped result still rounds to zero in the cast.
-__device__ __forceinline__ float exp2_poly(float x)
-{
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
-    constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261115f, c3 = 0.05517177f;
-    x = fmaxf(x, -16.0f);
-    const float t = x + kRound;
-    const float f = x - (t - kRound);
-    const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, c0);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// Two exp2_poly evaluations with the floating-point steps packed in pairs (f32x2).
-__device__ __forceinline__ void exp2_poly2(float &r0, float &r1, float x0, float x1)
-{
-    constexpr float kRound = 12582912.0f;
-    constexpr float c0 = 0.99992806f, c1 = 0.69326097f, c2 = 0.24261115f, c3 = 0.05517177f;
-    x0 = fmaxf(x0, -16.0f);
-    x1 = fmaxf(x1, -16.0f);
-    float t0, t1, n0, n1, f0, f1, p0, p1;
-    fma2(t0, t1, x0, x1, 1.0f, 1.0f, kRound, kRound);     // t = x + 1.5*2^23
-    fma2(n0, n1, t0, t1, 1.0f, 1.0f, -kRound, -kRound);   // n = round(x)
-    fma2(f0, f1, n0, n1, -1.0f, -1.0f, x0, x1);           // f = x - n
-    fma2(p0, p1, f0, f1, c3, c3, c2, c2);
-    fma2(p0, p1, p0, p1, f0, f1, c1, c1);
-    fma2(p0, p1, p0, p1, f0, f1, c0, c0);
-    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 // max of three floats in one instruction (sm_100a)
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {

@@ -262,11 +262,6 @@ sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, 
  * status word and returns.  Exercises the failure path without faulting the GPU. */
 sa_status sa_debug_wait_timeout(int timeout_us, void *stream);
 
-/* Debug: y[i] = 2^x[i] computed by the attention kernel's polynomial exponential (the
- * share of softmax exponentials moved off the MUFU pipe): Cody-Waite reduction and a
- * fitted cubic, max relative error 7.5e-5 for -16 <= x <= 9; inputs below -16 are
- * clamped to -16.  x, y: device fp32 [n]. */
-sa_status sa_debug_exp2_poly(const float *x, float *y, int n, void *stream);
 
 /* Synchronises the current device, returns and clears its device status word
  * (SA_OK or SA_ERR_DEVICE_TIMEOUT), or SA_ERR_CUDA if synchronisation failed. */
@@ -278,6 +273,16 @@ const char *sa_status_string(sa_status s);
 /* Bytes of library workspace sa_attn_fwd needs for this problem size, d = 128 or 64 (0 on
  * bad sizes).  Causal calls with a keep mask add B * H * ceil(N/128) * ceil(N/64) bytes. */
 size_t sa_workspace_bytes(int B, int H, int N, int d);
+
+/* Measurement aid (no counterpart on the pages): the device's own 8-bit tensor-core rate,
+ * the denominator of the attention kernel's roofline.  Launches one CTA per SM; each
+ * issues `reps` chains of four tcgen05 MMAs of M = 128, N = 256, K = 32 (one K = 128
+ * contraction, the way the attention kernel issues them) from shared memory into tensor
+ * memory: kind 0 = kind::i8 (int8 x int8 -> int32), kind 1 = kind::f8f6f4 with e4m3
+ * operands (-> fp32).  The caller times the launch (e.g. with CUDA events on `stream`);
+ * it performs SMs * reps * 4 * 2*128*256*32 operations.  reps in [1, 2^20]; the final
+ * bounded wait reports through sa_get_device_status. */
+sa_status sa_debug_mma_peak(int kind, int reps, void *stream);
 
 /* Frees the current device's workspace (synchronises the device first). */
 sa_status sa_release_workspace(void);

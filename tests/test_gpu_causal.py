@@ -75,3 +75,34 @@ def test_causal_full_size_480p(oracle, libsa, cuda_ok):
     got = gpu_rows(o, rows)
     assert np.abs(got - ref).max() <= O_MAX_ABS
     assert cosine(got, ref) >= O_MIN_COS
+
+
+def test_masked_out_zero_scale_block_leaves_the_max(oracle, libsa, cuda_ok):
+    """A step whose keys all come after the row (tile 0 in its pair's second step) must not
+    raise the row maximum, even where those key blocks have scale 0.  Keys 128-255 are zero
+    and the other keys are +8 / -8 rows that cancel, so the K mean is exactly 0 and blocks 2
+    and 3 quantise to scale 0; tile 0's queries are -8, so its real logits are about -720.
+    A maximum of 0 taken from the masked blocks would scale O and its row sum by e^-720 = 0
+    and return zeros.  Both kernels: no mask (two-tile kernel) and all blocks kept."""
+    from bit_quantized_attention_sa_b200.workloads import f32_to_bf16_bits
+    B, H, N = 1, 1, 512
+    rng = np.random.default_rng(161)
+    q = rng.standard_normal((B, H, N, 128)).astype(np.float32)
+    q[:, :, :128] = -8.0
+    k = np.zeros((B, H, N, 128), np.float32)
+    k[:, :, 0:128] = 8.0
+    k[:, :, 256:384] = -8.0
+    v = rng.standard_normal((B, H, N, 128)).astype(np.float32)
+    qb, kb, vb = f32_to_bf16_bits(q), f32_to_bf16_bits(k), f32_to_bf16_bits(v)
+    qk = oracle.quantize_qk(qb, kb)
+    assert np.all(qk[4] == 0) and np.all(qk[3][0, 0, 2:4] == 0)  # K mean 0; blocks 2, 3 scale 0
+    rows = [(0, r) for r in (0, 1, 63, 64, 100, 127, 128, 200, 255, 256, 400, 511)]
+    ref = oracle.attn_rows(qk, oracle.quantize_v(vb), N, sm_scale(), rows, None, 2, causal=True)
+    assert np.abs(ref[:6]).max() > 0.05  # the tile-0 rows are far from zero
+    qd, kd, vd = to_dev_bf16(qb), to_dev_bf16(kb), to_dev_bf16(vb)
+    ones = torch.ones((B, H, N // 128, N // 64), dtype=torch.uint8, device="cuda")
+    for o in (libsa.sa_attn_fwd_causal(qd, kd, vd), libsa.sa_attn_fwd_causal(qd, kd, vd, block_mask=ones)):
+        assert libsa.sa_get_device_status() == 0
+        got = gpu_rows(o, rows)
+        assert np.abs(got - ref).max() <= O_MAX_ABS
+        assert cosine(got, ref) >= O_MIN_COS
