@@ -294,15 +294,20 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             // ------------------------------------------------------------ producer
             bool ok = true;
             uint32_t g = 0, pl = 0;
+            // K/V tiles are read by every CTA working on the head: keep them in L2 in
+            // preference to the Q tiles, which one CTA reads once (DRAM traffic per launch at
+            // 40 x 75600: 2.43 GB with the hints, 2.49 GB without; 1.94 GB algorithmic)
+            const uint64_t pol_kv = l2_policy_evict_last(), pol_q = l2_policy_evict_first();
             for (int r = 0, p = item(0); p < npairs; p = item(++r), ++pl) {
                 const int bh = pair_head(p), qa = pair_qa(p);
                 const bool hasb = qa + 1 < nq;
                 if (pl >= 1 && ok) ok = mbar_wait(bar(kBarQEmpty), (pl - 1) & 1, abort_flag);
                 if (ok) {
                     mbar_arrive_expect_tx(bar(kBarQFull), (hasb ? 2u : 1u) * kQTileBytes);
-                    tma_load_2d(sbase + kOffQ, &tm_q, bar(kBarQFull), 0, bh * Npad + qa * 128);
+                    tma_load_2d_hint(sbase + kOffQ, &tm_q, bar(kBarQFull), 0, bh * Npad + qa * 128, pol_q);
                     if (hasb)
-                        tma_load_2d(sbase + kOffQ + kQTileBytes, &tm_q, bar(kBarQFull), 0, bh * Npad + qa * 128 + 128);
+                        tma_load_2d_hint(sbase + kOffQ + kQTileBytes, &tm_q, bar(kBarQFull), 0,
+                                         bh * Npad + qa * 128 + 128, pol_q);
                 }
                 const int ns = pair_steps(qa);
                 for (int j = 0; j < ns && ok; ++j, ++g) {
@@ -313,11 +318,13 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                     const uint32_t kb = sbase + kOffK + st * kKTileBytes;
                     const uint32_t vb = sbase + kOffV + st * 2 * kVHalfBytes;
                     mbar_arrive_expect_tx(bar(kBarKvFull + st), (two ? 2u : 1u) * (kKHalfBytes + kVHalfData));
-                    tma_load_2d(kb, &tm_k, bar(kBarKvFull + st), 0, bh * Npad + 128 * j);
-                    tma_load_2d(vb, &tm_v, bar(kBarKvFull + st), 128 * j, bh * 128);
+                    tma_load_2d_hint(kb, &tm_k, bar(kBarKvFull + st), 0, bh * Npad + 128 * j, pol_kv);
+                    tma_load_2d_hint(vb, &tm_v, bar(kBarKvFull + st), 128 * j, bh * 128, pol_kv);
                     if (two) {
-                        tma_load_2d(kb + kKHalfBytes, &tm_k, bar(kBarKvFull + st), 0, bh * Npad + 128 * j + 64);
-                        tma_load_2d(vb + kVHalfBytes, &tm_v, bar(kBarKvFull + st), 128 * j + 64, bh * 128);
+                        tma_load_2d_hint(kb + kKHalfBytes, &tm_k, bar(kBarKvFull + st), 0, bh * Npad + 128 * j + 64,
+                                         pol_kv);
+                        tma_load_2d_hint(vb + kVHalfBytes, &tm_v, bar(kBarKvFull + st), 128 * j + 64, bh * 128,
+                                         pol_kv);
                     }
                 }
             }
