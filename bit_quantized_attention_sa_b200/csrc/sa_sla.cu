@@ -21,8 +21,9 @@
 //   sla_state_sum_kernel  A_i = sum of the marginal blocks' states, for 16 query blocks at a
 //                         time (each H_j chunk is read once for all 16 rows of classes).
 //   sla_apply_kernel      one CTA per (head, 128-query block): phi(Q_i) A_i in shared memory,
-//                         division by the normaliser column, the projection, and the store
-//                         (fp32 out, or added to the bf16 output of the sparse part).
+//                         division by the normaliser column, the projection, and the fp32
+//                         store.  The SLA forward hands that fp32 output to the attention
+//                         kernel's epilogue, which adds it before the one bf16 rounding.
 //   sla_critical_kernel   the keep mask (class >= 2) of the sparse part.
 #include <cstdint>
 #include <cuda_bf16.h>
