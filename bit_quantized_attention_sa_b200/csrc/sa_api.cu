@@ -54,6 +54,21 @@ bool encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint6
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_tmap_3d_f32(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                        CUtensorMapSwizzle swizzle)
+{
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+    const cuuint32_t box[3] = {box0, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ validation
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -595,12 +610,11 @@ sa_status sa_sla_linear(const void *q, const void *k, const void *v, const uint8
     if ((r = check_sla(s, phi, {q, k, v, out})) != SA_OK) return r;
     if (proj && (r = check_ptrs({proj})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
-    const size_t sb = align256(sla_state_bytes(s));
     WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(lock, sb + sla_sum_bytes(s), &ws)) != SA_OK) return r;
-    return launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws),
-                             reinterpret_cast<float *>(ws + sb), out, static_cast<cudaStream_t>(stream)) == cudaSuccess
+    if ((r = get_workspace(lock, sla_workspace_bytes(s), &ws)) != SA_OK) return r;
+    return launch_sla_linear(q, k, v, classes, s, phi, proj, ws, out, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
                ? SA_OK
                : SA_ERR_CUDA;
 }
@@ -615,22 +629,21 @@ sa_status sa_sla_fwd(const void *q, const void *k, const void *v, void *o, int B
     if ((r = check_sla(s, phi, {q, k, v, o})) != SA_OK) return r;
     if (proj && (r = check_ptrs({proj})) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
-    // workspace: [attention prologue | keep mask | states | summed states | linear part, fp32]
+    // workspace: [attention prologue | keep mask | linear-branch states | linear part, fp32]
     const size_t attn = align256(ws_layout(s).total);
     const size_t nmask = size_t(s.BH()) * size_t(s.nq()) * size_t(s.nk());
-    const size_t mb = align256(nmask), sb = align256(sla_state_bytes(s)), ub = align256(sla_sum_bytes(s));
+    const size_t mb = align256(nmask), sb = align256(sla_workspace_bytes(s));
     const size_t lb = size_t(s.BH()) * size_t(s.N) * kD * sizeof(float);
     WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(lock, attn + mb + sb + ub + lb, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, attn + mb + sb + lb, &ws)) != SA_OK) return r;
     uint8_t *keep = ws + attn;
-    float *lin = reinterpret_cast<float *>(ws + attn + mb + sb + ub);
+    float *lin = reinterpret_cast<float *>(ws + attn + mb + sb);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (launch_sla_critical(classes, int64_t(nmask), keep, st) != cudaSuccess) return SA_ERR_CUDA;
     // the linear part first, in fp32; the sparse part's epilogue adds it to O before O's
     // only rounding to bf16
-    if (launch_sla_linear(q, k, v, classes, s, phi, proj, reinterpret_cast<float *>(ws + attn + mb),
-                          reinterpret_cast<float *>(ws + attn + mb + sb), lin, st) != cudaSuccess)
+    if (launch_sla_linear(q, k, v, classes, s, phi, proj, ws + attn + mb, lin, st) != cudaSuccess)
         return SA_ERR_CUDA;
     return attn_fwd_device(q, k, v, o, s, sm_scale, keep, st, false, lin);
 }
@@ -738,11 +751,11 @@ sa_status sa_debug_mma_peak(int kind, int reps, void *stream)
 
 sa_status sa_get_device_status(void)
 {
-    int st = 0, st_w8a8 = 0, st_peak = 0;
+    int st = 0, st_w8a8 = 0, st_peak = 0, st_sla = 0;
     if (read_and_clear_status(&st) != cudaSuccess || read_and_clear_w8a8_status(&st_w8a8) != cudaSuccess ||
-        read_and_clear_peak_status(&st_peak) != cudaSuccess)
+        read_and_clear_peak_status(&st_peak) != cudaSuccess || read_and_clear_sla_status(&st_sla) != cudaSuccess)
         return SA_ERR_CUDA;
-    return st == 0 && st_w8a8 == 0 && st_peak == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
+    return st == 0 && st_w8a8 == 0 && st_peak == 0 && st_sla == 0 ? SA_OK : SA_ERR_DEVICE_TIMEOUT;
 }
 
 const char *sa_status_string(sa_status s)

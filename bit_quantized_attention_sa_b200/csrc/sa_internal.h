@@ -76,14 +76,16 @@ cudaError_t launch_w8a8_gemm(const CUtensorMap &tm_x, const CUtensorMap &tm_w, c
                              const float *sw, int M, int N, int nkb, void *y, cudaStream_t st);
 cudaError_t read_and_clear_w8a8_status(int *status);
 // ---- SLA linear branch (sa_sla.cu)
-size_t sla_state_bytes(const Shape &s);  // per-key-block states, fp32
-size_t sla_sum_bytes(const Shape &s);    // per-query-block summed states, fp32
+// Workspace of launch_sla_linear: the per-key-block and per-query-block states of one group
+// of heads (fp32), at most about 1 GiB whatever the number of heads.
+size_t sla_workspace_bytes(const Shape &s);
 // The branch for all rows: fp32 out [B,H,N,d].  classes uint8 [B,H,nq,nk] (1 = marginal);
-// proj fp32 [d][d] or null.
+// proj fp32 [d][d] or null; workspace of sla_workspace_bytes(s) bytes, 256-byte aligned.
 cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, const Shape &s,
-                              int phi, const float *proj, float *state, float *sums, float *out, cudaStream_t st);
+                              int phi, const float *proj, void *workspace, float *out, cudaStream_t st);
 // keep[e] = classes[e] >= 2 (the sparse part's block mask), n entries.
 cudaError_t launch_sla_critical(const uint8_t *classes, int64_t n, uint8_t *keep, cudaStream_t st);
+cudaError_t read_and_clear_sla_status(int *status);
 // Reads and clears the device status word of the current device (synchronous).
 cudaError_t read_and_clear_status(int *status);
 // ---- measured tensor-core peak (sa_peak.cu): one CTA per SM, reps chains of four
@@ -95,5 +97,9 @@ cudaError_t read_and_clear_peak_status(int *status);
 bool encode_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
                        uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                        CUtensorMapSwizzle swizzle);
+// fp32 [d2][d1][d0] (d0 contiguous), box {box0, box1, 1}, zero fill
+bool encode_tmap_3d_f32(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t box0, uint32_t box1,
+                        CUtensorMapSwizzle swizzle);
 
 }  // namespace sa

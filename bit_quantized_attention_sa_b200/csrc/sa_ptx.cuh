@@ -98,6 +98,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// 3-D tiled bulk tensor load global -> shared.  The innermost coordinate x times the
+// element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint32_t bar, int x, int y, int z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 // The same with an L2 eviction-priority policy (from createpolicy) for the loaded lines.
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void *tmap, uint32_t bar, int x, int y,
                                                  uint64_t policy)
@@ -189,6 +200,19 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
+// D(tmem) (+)= A(smem desc) * B(smem desc)^T, TF32 operands (32-bit containers whose low
+// 13 mantissa bits the tensor core does not use), fp32 accumulator.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Instruction descriptor fields (dense, no negation, both operands K-major):
 //   [4,6) accumulator format (1 = f32, 2 = s32); [7,10) A format; [10,13) B format;
 //   [17,23) N >> 3; [24,29) M >> 4.
@@ -201,6 +225,13 @@ __host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N)
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
 {
     return (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(N >> 3) << 17) |
+           (uint32_t(M >> 4) << 24);
+}
+// kind::tf32 (operand format 2), fp32 accumulator; bit 15 set: A is MN-major (M
+// contiguous in shared memory), B stays K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32_amn(int M, int N)
+{
+    return (1u << 4) | (2u << 7) | (2u << 10) | (1u << 15) | (uint32_t(N >> 3) << 17) |
            (uint32_t(M >> 4) << 24);
 }
 
@@ -218,6 +249,23 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t sbo_bytes, ui
     d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= uint64_t(1) << 46;
     d |= uint64_t(layout) << 61;
+    return d;
+}
+
+// Descriptor of an MN-major 32-bit (TF32) operand.  Such operands take the 128-byte
+// swizzle with 32-byte granules (layout 1): an atom is 4 rows along K of 128 bytes along M
+// (or N), the four 32-byte granules of row r stored at granule position g ^ (r & 3) -- the
+// pattern TMA writes with CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B.  Atoms follow each other
+// along M at lbo_bytes and along K at sbo_bytes.
+enum : uint32_t { SWZ_128B_BASE32B = 1 };
+__device__ __forceinline__ uint64_t sdesc_mn32(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes)
+{
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1) << 46;
+    d |= uint64_t(SWZ_128B_BASE32B) << 61;
     return d;
 }
 

@@ -29,16 +29,13 @@
 #include <cuda_bf16.h>
 
 #include "sa_internal.h"
+#include "sa_ptx.cuh"
 
 namespace sa {
 namespace {
 
 constexpr int kStateCols = 136;                      // H_j columns, then Z_j, then zeros
 constexpr int kStateFloats = kD * kStateCols;        // 17408 per key (or query) block
-constexpr int kSumChunk = 1024;                      // floats of a state per sum CTA
-constexpr int kSumChunks = kStateFloats / kSumChunk;  // 17
-constexpr int kSumGroup = 16;                        // query blocks per sum CTA
-static_assert(kStateFloats % kSumChunk == 0, "state chunks");
 
 // phi of one 128-feature row held by a warp, 4 features per lane (features 4 lane .. +3).
 __device__ __forceinline__ void phi_row_warp(float (&x)[4], int phi)
@@ -134,57 +131,212 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// grid (kSumChunks, ceil(nq / 16), BH), 256 threads; dynamic shared memory nk uint32.
-// A_i (chunk) = sum over j ascending of the states of the blocks with classes[i][j] == 1.
-__global__ void __launch_bounds__(256)
-    sla_state_sum_kernel(const float *__restrict__ state, const uint8_t *__restrict__ classes, int nq, int nk,
-                         float *__restrict__ sums)
+// ---- the class-weighted state sum on the tensor cores
+// D[n][i] = sum_j H[j][n] C[i][j] with C[i][j] = (classes[i][j] == 1), for one head: the
+// GEMM of the states (K = key blocks j, M = the 17408 state entries n) with the 0/1 class
+// rows of up to 256 query blocks i (N).  kind::tf32 with fp32 accumulation in tensor
+// memory.  C is exact in TF32; the states are split in shared memory into hi (the top 11
+// significant bits, exact in TF32) and lo = H - hi (exact in fp32, of which the tensor core
+// uses the top 11 bits), and both halves are multiplied, so every product carries about 22
+// significant bits of H: far below fp32 accumulation error relative to the 1e-4 bound.
+//
+// One CTA per (query-block tile, 128 state entries, head), query-block tiles fastest so
+// that the CTAs reading one chunk of states run together and share it through L2.
+//   warps 0-3  per k-block of 32 key blocks: split the landed state tile into hi and lo;
+//              then the epilogue (warp w owns tensor-memory lanes 32w .. 32w+31, i.e. state
+//              entries n0 + 32w + lane).
+//   warp 4     TMA producer: the state tile, 4 boxes of 32 entries x 32 key blocks, in the
+//              MN-major layout with 32-byte swizzle granules that TF32 operands need; and
+//              the tile of C (fp32 0/1, written once per call by sla_marginal_kernel),
+//              K-major with the usual 128-byte swizzle.
+//   warp 5     MMA issuer: per k-block, 4 steps of K = 8, each hi and lo.
+namespace summ {
+constexpr int kM = 128;        // state entries per tile (MMA M)
+constexpr int kKb = 32;        // key blocks per k-block: 128 bytes of fp32
+constexpr int kStages = 3;
+constexpr int kMaxNT = 256;    // query blocks per tile (MMA N)
+constexpr int kThreads = 192;
+constexpr int kWarpTma = 4, kWarpMma = 5;
+constexpr uint32_t kABytes = kM * kKb * 4;      // 16 KB: 4 atoms of 32 entries x 32 rows
+constexpr uint32_t kBBytes = kMaxNT * kKb * 4;  // 32 KB
+constexpr uint32_t kOffAhi = 0;
+constexpr uint32_t kOffAlo = kOffAhi + kStages * kABytes;
+constexpr uint32_t kOffB = kOffAlo + kStages * kABytes;
+constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
+constexpr int kBarFull = 0, kBarEmpty = kStages, kBarReady = 2 * kStages, kBarAcc = 3 * kStages;
+constexpr uint32_t kOffMisc = kOffBar + 8 * (3 * kStages + 1);
+constexpr uint32_t kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte alignment
+static_assert(kOffB % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0, "swizzle atoms");
+static_assert(kSmem <= 232448, "shared memory");
+}  // namespace summ
+
+__device__ int g_sla_status;  // 0 = OK, 6 = a bounded wait expired
+
+// A wait bounded by time alone (not by the abort flag): used to let this CTA's own
+// copies and MMAs land before it frees its memory.
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity)
 {
-    extern __shared__ uint32_t marg_bits[];  // bit g: query block i0 + g has class 1 at j
-    const int64_t bh = blockIdx.z;
-    const int cc = blockIdx.x, i0 = blockIdx.y * kSumGroup, tid = threadIdx.x;
-    const int ng = min(kSumGroup, nq - i0);
-    for (int j = tid; j < nk; j += blockDim.x) {
-        uint32_t bits = 0;
-        for (int g = 0; g < ng; ++g) bits |= uint32_t(classes[(bh * nq + i0 + g) * int64_t(nk) + j] == 1) << g;
-        marg_bits[j] = bits;
-    }
-    __syncthreads();
-    float4 acc[kSumGroup];
-#pragma unroll
-    for (int g = 0; g < kSumGroup; ++g) acc[g] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    const float *src = state + bh * int64_t(nk) * kStateFloats + cc * kSumChunk + 4 * tid;
-    // 8 key blocks per step: their loads are all in flight before the first is added
-    constexpr int kAhead = 8;
-    for (int j0 = 0; j0 < nk; j0 += kAhead) {
-        uint32_t bits[kAhead];
-        float4 h[kAhead];
-#pragma unroll
-        for (int u = 0; u < kAhead; ++u) {
-            bits[u] = j0 + u < nk ? marg_bits[j0 + u] : 0u;
-            h[u] = bits[u] ? __ldg(reinterpret_cast<const float4 *>(src + int64_t(j0 + u) * kStateFloats))
-                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > SA_WAIT_LIMIT_NS) return false;
+    return true;
+}
+
+// grid (ceil(nq / nt), 17408 / 128, BH), summ::kThreads threads, summ::kSmem bytes.
+// nt: query blocks per tile, a multiple of 16 in [16, 256].
+__global__ void __launch_bounds__(summ::kThreads, 1)
+    sla_sum_mma_kernel(const __grid_constant__ CUtensorMap tm_state, const __grid_constant__ CUtensorMap tm_c,
+                       int nq, int nk, int nt, float *__restrict__ sums)
+{
+    using namespace summ;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i0 = blockIdx.x * nt, n0 = blockIdx.y * kM, bh = blockIdx.z;
+    const int nkb = (nk + kKb - 1) / kKb;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    auto bar = [&](int i) -> uint32_t { return sbase + kOffBar + 8u * uint32_t(i); };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar(kBarFull + s), 1);
+            mbar_init(bar(kBarEmpty + s), 1);
+            mbar_init(bar(kBarReady + s), 4);
         }
-        // keeps the compiler from sinking each load to its first use
+        mbar_init(bar(kBarAcc), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == kWarpMma) tmem_alloc(sbase + kOffMisc, kMaxNT);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kWarpTma) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_state);
+            prefetch_tmap(&tm_c);
+            bool ok = true;
+            int kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = kb % kStages;
+                if (kb >= kStages) ok = mbar_wait(bar(kBarEmpty + s), ((kb / kStages) & 1) ^ 1, abort_flag);
+                if (!ok) break;
+                const uint32_t dst = sbase + kOffAhi + uint32_t(s) * kABytes;
+                mbar_arrive_expect_tx(bar(kBarFull + s), kABytes + uint32_t(nt) * 128u);
 #pragma unroll
-        for (int u = 0; u < kAhead; ++u) asm volatile("" ::"f"(h[u].x), "f"(h[u].y), "f"(h[u].z), "f"(h[u].w));
-#pragma unroll
-        for (int u = 0; u < kAhead; ++u) {
-#pragma unroll
-            for (int g = 0; g < kSumGroup; ++g) {
-                if ((bits[u] >> g) & 1u) {
-                    acc[g].x += h[u].x;
-                    acc[g].y += h[u].y;
-                    acc[g].z += h[u].z;
-                    acc[g].w += h[u].w;
-                }
+                for (int c = 0; c < kM / 32; ++c)
+                    tma_load_3d(dst + 4096u * c, &tm_state, bar(kBarFull + s), n0 + 32 * c, kb * kKb, bh);
+                tma_load_3d(sbase + kOffB + uint32_t(s) * kBBytes, &tm_c, bar(kBarFull + s), kb * kKb, i0, bh);
+            }
+            // the last loads issued have landed before the CTA's memory is released
+            bool drained = true;
+            for (int d = kb > kStages ? kb - kStages : 0; d < kb; ++d)
+                drained = drain_wait(bar(kBarFull + d % kStages), (d / kStages) & 1) && drained;
+            if (!ok || !drained) {
+                *abort_flag = 1;
+                atomicExch(&g_sla_status, 6);
             }
         }
-    }
-    float *dst = sums + (bh * nq + i0) * int64_t(kStateFloats) + cc * kSumChunk + 4 * tid;
+    } else if (warp == kWarpMma) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_tf32_f32_amn(kM, nt);
+            bool ok = true;
+            int kb = 0;
+            for (; kb < nkb; ++kb) {
+                const int s = kb % kStages;
+                ok = mbar_wait(bar(kBarReady + s), (kb / kStages) & 1, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t ahi = sbase + kOffAhi + uint32_t(s) * kABytes;
+                const uint32_t alo = sbase + kOffAlo + uint32_t(s) * kABytes;
+                const uint32_t bt = sbase + kOffB + uint32_t(s) * kBBytes;
 #pragma unroll
-    for (int g = 0; g < kSumGroup; ++g)
-        if (g < ng) *reinterpret_cast<float4 *>(dst + int64_t(g) * kStateFloats) = acc[g];
+                for (int kk = 0; kk < kKb / 8; ++kk) {
+                    // A: rows 8kk .. 8kk+7 (two 4-row atoms, 512 bytes apart) of each column
+                    // of 32 entries, the columns 4096 bytes apart; B: 32 bytes of K per step
+                    const uint64_t bdesc = sdesc(bt + 32u * kk, 1024, SWZ_128B);
+                    mma_tf32(tmem, sdesc_mn32(ahi + 1024u * kk, 4096, 512), bdesc, idesc, (kb | kk) != 0);
+                    mma_tf32(tmem, sdesc_mn32(alo + 1024u * kk, 4096, 512), bdesc, idesc, 1);
+                }
+                tc_commit(bar(kBarEmpty + s));
+            }
+            if (ok) tc_commit(bar(kBarAcc));
+            // this thread's MMAs have completed before the tensor memory is freed
+            if (kb > 0 && !drain_wait(bar(kBarEmpty + (kb - 1) % kStages), ((kb - 1) / kStages) & 1)) ok = false;
+            if (!ok) {
+                *abort_flag = 1;
+                atomicExch(&g_sla_status, 6);
+            }
+        }
+    } else {
+        // ---- warps 0-3: the hi/lo split, then the epilogue.  The full barrier of a stage
+        // completes only after the producer's wait for that stage's previous MMAs, so the
+        // lo tile is free to overwrite once the loads have landed.
+        bool ok = true;
+        for (int kb = 0; kb < nkb && ok; ++kb) {
+            const int s = kb % kStages;
+            ok = mbar_wait(bar(kBarFull + s), (kb / kStages) & 1, abort_flag);
+            if (!ok) break;
+            // hi keeps the sign, exponent and top 10 mantissa bits; lo = H - hi exactly
+            float4 *ahi = reinterpret_cast<float4 *>(smem + kOffAhi + uint32_t(s) * kABytes);
+            float4 *alo = reinterpret_cast<float4 *>(smem + kOffAlo + uint32_t(s) * kABytes);
+#pragma unroll
+            for (int u = 0; u < int(kABytes / 16) / 128; ++u) {
+                const int e = threadIdx.x + 128 * u;
+                const float4 x = ahi[e];
+                float4 h;
+                h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+                h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+                h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+                h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
+                ahi[e] = h;
+                alo[e] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarReady + s));
+        }
+        if (ok) ok = mbar_wait(bar(kBarAcc), 0, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+            tc_fence_after();
+            const int n = n0 + 32 * warp + lane;
+            float *dst = sums + int64_t(bh) * nq * int64_t(kStateFloats) + n;
+            for (int c0 = 0; c0 < nt; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32_wait(tmem + (uint32_t(32 * warp) << 16) + uint32_t(c0), r);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int i = i0 + c0 + c;
+                    if (c0 + c < nt && i < nq) dst[int64_t(i) * kStateFloats] = __uint_as_float(r[c]);
+                }
+            }
+        } else if (lane == 0) {
+            *abort_flag = 1;
+            atomicExch(&g_sla_status, 6);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpMma) tmem_dealloc(tmem, kMaxNT);
+}
+
+// C of the state sum: cm[bh][i][j] = (classes[bh][i][j] == 1) as fp32, for j < nk4 (a
+// multiple of 4, so that rows are 16-byte aligned for TMA); zero for j >= nk.
+__global__ void sla_marginal_kernel(const uint8_t *__restrict__ classes, int64_t rows, int nk, int nk4,
+                                    float *__restrict__ cm)
+{
+    const int64_t n = rows * nk4;
+    for (int64_t e = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+        const int64_t r = e / nk4;
+        const int j = int(e - r * nk4);
+        cm[e] = (j < nk && classes[r * nk + j] == 1) ? 1.0f : 0.0f;
+    }
 }
 
 // Shared memory of the apply kernel (floats): phi(Q) [128][132] (row-padded), then the
@@ -309,11 +461,33 @@ __global__ void sla_critical_kernel(const uint8_t *__restrict__ classes, int64_t
 
 }  // namespace
 
-size_t sla_state_bytes(const Shape &s) { return size_t(s.BH()) * size_t(s.nk()) * kStateFloats * sizeof(float); }
-size_t sla_sum_bytes(const Shape &s) { return size_t(s.BH()) * size_t(s.nq()) * kStateFloats * sizeof(float); }
+// The branch runs over groups of heads whose states and summed states together take at
+// most kChunkBudget bytes (at least one head per group), so its workspace does not grow
+// with the number of heads.
+constexpr size_t kChunkBudget = size_t(1) << 30;
+
+static size_t head_state_bytes(const Shape &s) { return size_t(s.nk()) * kStateFloats * sizeof(float); }
+static size_t head_sum_bytes(const Shape &s) { return size_t(s.nq()) * kStateFloats * sizeof(float); }
+static int nk4_of(const Shape &s) { return int((s.nk() + 3) / 4 * 4); }
+static size_t head_c_bytes(const Shape &s) { return size_t(s.nq()) * size_t(nk4_of(s)) * sizeof(float); }
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static int64_t chunk_heads(const Shape &s)
+{
+    const int64_t per = int64_t(head_state_bytes(s) + head_sum_bytes(s) + head_c_bytes(s));
+    const int64_t g = int64_t(kChunkBudget) / per;
+    return g < 1 ? 1 : (g > s.BH() ? s.BH() : g);
+}
+
+// workspace: [states | summed states | C], each for chunk_heads(s) heads
+size_t sla_workspace_bytes(const Shape &s)
+{
+    const size_t g = size_t(chunk_heads(s));
+    return up256(g * head_state_bytes(s)) + up256(g * head_sum_bytes(s)) + g * head_c_bytes(s);
+}
 
 cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const uint8_t *classes, const Shape &s,
-                              int phi, const float *proj, float *state, float *sums, float *out, cudaStream_t st)
+                              int phi, const float *proj, void *workspace, float *out, cudaStream_t st)
 {
     static bool attr_set[64] = {false};
     int dev = 0;
@@ -323,24 +497,58 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
         if ((e = cudaFuncSetAttribute(sla_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(state_smem))) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(sla_state_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(sizeof(uint32_t) * kMaskMaxKeyBlocks))) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(sla_sum_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(summ::kSmem))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(kApplySmemBytes))) != cudaSuccess)
             return e;
         attr_set[dev] = true;
     }
-    const int nq = int(s.nq()), nk = int(s.nk()), N = int(s.N);
-    const auto *qb = static_cast<const uint16_t *>(q);
-    sla_state_kernel<<<dim3(unsigned(nk), unsigned(s.BH())), 256, state_smem, st>>>(
-        static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(v), N, nk, phi, state);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    sla_state_sum_kernel<<<dim3(unsigned(kSumChunks), unsigned((nq + kSumGroup - 1) / kSumGroup), unsigned(s.BH())),
-                           256, sizeof(uint32_t) * size_t(nk), st>>>(state, classes, nq, nk, sums);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const dim3 ga(unsigned(nq), unsigned(s.BH()));
-    sla_apply_kernel<<<ga, 256, kApplySmemBytes, st>>>(qb, sums, proj, N, nq, phi, out);
-    return cudaGetLastError();
+    const int nq = int(s.nq()), nk = int(s.nk()), N = int(s.N), nk4 = nk4_of(s);
+    const int64_t G = chunk_heads(s), tok = int64_t(N) * kD;
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    float *state = reinterpret_cast<float *>(w);
+    float *sums = reinterpret_cast<float *>(w + up256(size_t(G) * head_state_bytes(s)));
+    float *cm = reinterpret_cast<float *>(w + up256(size_t(G) * head_state_bytes(s)) +
+                                          up256(size_t(G) * head_sum_bytes(s)));
+    // query-block tiles of nt <= 256 (a multiple of 16), as even as the count allows
+    const int ntiles = (nq + summ::kMaxNT - 1) / summ::kMaxNT;
+    const int nt = ((nq + ntiles - 1) / ntiles + 15) / 16 * 16;
+    for (int64_t h0 = 0; h0 < s.BH(); h0 += G) {
+        const int64_t g = s.BH() - h0 < G ? s.BH() - h0 : G;
+        sla_state_kernel<<<dim3(unsigned(nk), unsigned(g)), 256, state_smem, st>>>(
+            static_cast<const uint16_t *>(k) + h0 * tok, static_cast<const uint16_t *>(v) + h0 * tok, N, nk, phi,
+            state);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int64_t crows = g * nq, celems = crows * nk4;
+        const int cblocks = int(celems / 1024 + 1 < 4096 ? celems / 1024 + 1 : 4096);
+        sla_marginal_kernel<<<cblocks, 256, 0, st>>>(classes + h0 * nq * int64_t(nk), crows, nk, nk4, cm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        CUtensorMap tm_state, tm_c;
+        if (!encode_tmap_3d_f32(&tm_state, state, kStateFloats, uint64_t(nk), uint64_t(g),
+                                uint64_t(kStateFloats) * sizeof(float), head_state_bytes(s), 32, summ::kKb,
+                                CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
+            !encode_tmap_3d_f32(&tm_c, cm, uint64_t(nk4), uint64_t(nq), uint64_t(g), uint64_t(nk4) * sizeof(float),
+                                head_c_bytes(s), summ::kKb, uint32_t(nt), CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        sla_sum_mma_kernel<<<dim3(unsigned((nq + nt - 1) / nt), unsigned(kStateFloats / summ::kM), unsigned(g)),
+                             summ::kThreads, summ::kSmem, st>>>(tm_state, tm_c, nq, nk, nt, sums);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        sla_apply_kernel<<<dim3(unsigned(nq), unsigned(g)), 256, kApplySmemBytes, st>>>(
+            static_cast<const uint16_t *>(q) + h0 * tok, sums, proj, N, nq, phi, out + h0 * tok);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t read_and_clear_sla_status(int *status)
+{
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(status, g_sla_status, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_sla_status, &zero, sizeof(int));
 }
 
 cudaError_t launch_sla_critical(const uint8_t *classes, int64_t n, uint8_t *keep, cudaStream_t st)

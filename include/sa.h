@@ -234,9 +234,14 @@ sa_status sa_w8a8_linear(const void *x, const int8_t *w_codes, const float *w_sc
  * with phi = SA_PHI_SOFTMAX (softmax over the d features of a row) or SA_PHI_ELU1
  * (elu(x) + 1), projected by W: out[r][c] = sum_e W[c][e] O_lin[r][e], W fp32 [d][d]
  * (device; NULL = identity; in SLA a trained layer).  Evaluated in fp32 in the factorised
- * form phi(q)^T (sum_t phi(k_t) v_t^T) / (phi(q) . sum_t phi(k_t)).
- * Needs ceil(N/64) <= 4096 (else SA_ERR_UNSUPPORTED).  Uses the library workspace:
- * 69,632 bytes per 64-key block and per 128-query block of every head. */
+ * form phi(q)^T (sum_t phi(k_t) v_t^T) / (phi(q) . sum_t phi(k_t)): per 64-key block
+ * the state sum_t phi(k_t) [v_t, 1]^T (128 x 129), then per 128-query block the sum of
+ * its marginal blocks' states on the tensor cores (TF32 products of the 0/1 class matrix
+ * with the states split into two TF32 terms, about 22 significant bits each, fp32
+ * accumulation), then the division and projection.
+ * Needs ceil(N/64) <= 4096 (else SA_ERR_UNSUPPORTED).  Uses the library workspace for
+ * the states of one group of heads at a time: 69,632 bytes per 64-key block and per
+ * 128-query block of a head, at most about 1 GiB (one head at least). */
 enum { SA_PHI_SOFTMAX = 0, SA_PHI_ELU1 = 1 };
 
 /* The linear branch alone: out fp32 [B,H,N,d] (device, caller-owned) = W O_lin. */

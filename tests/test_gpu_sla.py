@@ -20,10 +20,13 @@ def _proj(seed, d=128):
 
 
 def _rows(B, H, N, per_head=6, seed=7):
-    return sample_rows(B, H, N, per_head, seed)
+    rows = sample_rows(B, H, N, per_head, seed)
+    if N > 32768:  # more than 256 query blocks: rows of the second query-block tile too
+        rows = rows + [(0, 32768 + 5), (B * H - 1, N - 1)]
+    return rows
 
 
-@pytest.mark.parametrize("B,H,N", [(1, 2, 1), (1, 2, 200), (2, 1, 1000), (1, 3, 3000)])
+@pytest.mark.parametrize("B,H,N", [(1, 2, 1), (1, 2, 200), (2, 1, 1000), (1, 3, 3000), (1, 2, 40000)])
 @pytest.mark.parametrize("phi", [0, 1])
 def test_linear_branch_matches_oracle(oracle, libsa, cuda_ok, B, H, N, phi):
     q, k, v, _ = make_inputs(B, H, N, seed=100 + N + phi, outliers=True)
