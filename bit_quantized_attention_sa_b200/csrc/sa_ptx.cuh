@@ -227,12 +227,12 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N)
     return (1u << 4) | (0u << 7) | (0u << 10) | (uint32_t(N >> 3) << 17) |
            (uint32_t(M >> 4) << 24);
 }
-// kind::tf32 (operand format 2), fp32 accumulator; bit 15 set: A is MN-major (M
-// contiguous in shared memory), B stays K-major.
-__host__ __device__ constexpr uint32_t idesc_tf32_f32_amn(int M, int N)
+// kind::tf32 (operand format 2), fp32 accumulator; bit 15 (16) set: A (B) is MN-major, M
+// (N) contiguous in shared memory, else K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N, bool a_mn, bool b_mn)
 {
-    return (1u << 4) | (2u << 7) | (2u << 10) | (1u << 15) | (uint32_t(N >> 3) << 17) |
-           (uint32_t(M >> 4) << 24);
+    return (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
+           (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 // Shared-memory matrix descriptor for a K-major operand in a swizzled layout:

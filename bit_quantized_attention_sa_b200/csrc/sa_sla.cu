@@ -13,18 +13,22 @@
 // quantised attention of the critical (class >= 2) blocks.  phi is the softmax over the
 // d features of a row, or elu + 1.
 //
-// Kernels (fp32 throughout):
-//   sla_state_kernel      one CTA per (head, 64-key block): H_j (128 x 128) and Z_j, stored
-//                         as one 128 x 136 block whose column 128 is Z_j (columns 129-135
-//                         zero), so that the apply step gets the normaliser from the same
-//                         product as the numerator.
-//   sla_state_sum_kernel  A_i = sum of the marginal blocks' states, for 16 query blocks at a
-//                         time (each H_j chunk is read once for all 16 rows of classes).
-//   sla_apply_kernel      one CTA per (head, 128-query block): phi(Q_i) A_i in shared memory,
-//                         division by the normaliser column, the projection, and the fp32
-//                         store.  The SLA forward hands that fp32 output to the attention
+// Kernels, over groups of heads whose states fit a bounded workspace:
+//   sla_state_kernel      one CTA per (head, 64-key block), fp32 on the CUDA cores: H_j
+//                         (128 x 128) and Z_j, stored as one 128 x 136 block whose column
+//                         128 is Z_j (columns 129-135 zero), so that the apply step gets the
+//                         normaliser from the same product as the numerator.
+//   sla_marginal_kernel   the 0/1 matrix C[i][j] = (class == 1) in fp32.
+//   sla_sum_mma_kernel    A_i = sum_j C[i][j] H_j for every query block: a TF32 tcgen05 GEMM
+//                         (K = key blocks) with the states split into hi + lo terms.
+//   sla_apply_mma_kernel  one CTA per (head, 128-query block): phi(Q_i) [A_i | z_i] and the
+//                         projection as TF32 tcgen05 GEMMs with both operands split into hi +
+//                         lo (three products each), the division by the normaliser between
+//                         them, fp32 out.  The SLA forward hands that output to the attention
 //                         kernel's epilogue, which adds it before the one bf16 rounding.
 //   sla_critical_kernel   the keep mask (class >= 2) of the sparse part.
+// The hi/lo splits carry about 22 significant bits into every product; accumulation is
+// fp32, so the branch stays within fp32-level error of the factorised form.
 #include <cstdint>
 #include <cuda_bf16.h>
 
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(summ::kThreads, 1)
         }
     } else if (warp == kWarpMma) {
         if (lane == 0) {
-            const uint32_t idesc = idesc_tf32_f32_amn(kM, nt);
+            const uint32_t idesc = idesc_tf32_f32(kM, nt, true, false);
             bool ok = true;
             int kb = 0;
             for (; kb < nkb; ++kb) {
@@ -339,118 +343,285 @@ __global__ void sla_marginal_kernel(const uint8_t *__restrict__ classes, int64_t
     }
 }
 
-// Shared memory of the apply kernel (floats): phi(Q) [128][132] (row-padded), then the
-// summed state [128][136]; W^T [128][132] reuses the phi(Q) region and O_lin [128][132]
-// the state region once they are consumed.
-constexpr int kApplyLd = 132;
-constexpr int kApplyPhi = 0, kApplyState = kD * kApplyLd, kApplyDen = kApplyState + kD * kStateCols;
-constexpr int kApplySmemFloats = kApplyDen + kD;
-constexpr size_t kApplySmemBytes = size_t(kApplySmemFloats) * sizeof(float);
+// ---- the apply step on the tensor cores
+// For one (head, 128-query block i):
+//   GEMM1  D1[r][b] = sum_a phi(q_r)[a] A_i[a][b]   (M = 128 rows, N = 144: the 128 value
+//          columns, the normaliser column 128 and zeros, K = 128 features)
+//   O_lin[r][f] = D1[r][f] / D1[r][128]  (0 when the normaliser is not positive)
+//   GEMM2  out[r][c] = sum_f O_lin[r][f] W[c][f]     (M = 128, N = 128, K = 128; skipped
+//          without a projection, when out = O_lin)
+// Both are kind::tf32 with both operands split into hi + lo and three products (hi*hi,
+// hi*lo, lo*hi), about 22 significant bits per product, fp32 accumulation in tensor memory.
+//   warps 0-3  thread r owns row r: phi(q_r) into the phi tiles, then O_lin from D1 into the
+//              O tiles, then out from D2 (tensor-memory lanes of warp w: 32w .. 32w+31).
+//   warps 4-7  split the A_i halves (TMA) into hi/lo; load W halves and split them.
+//   warp 8     lane 0 issues the TMA loads and the MMAs.
+// Shared memory: region R0 holds phi (hi, lo: 4 K-atoms of 128 rows x 128 bytes each) for
+// GEMM1 and then, per K half of GEMM2, the O and W tiles (hi, lo: 2 K-atoms each); region R1
+// holds one K half (64 features) of A_i (hi, lo), MN-major with 32-byte swizzle granules:
+// 5 columns of 32 entries x 64 rows.
+namespace appm {
+constexpr int kThreads = 288;
+constexpr int kWarpIssue = 8;
+constexpr uint32_t kAtom = 128 * 128;            // 128 rows x 128 bytes, K-major
+constexpr uint32_t kOffPhiHi = 0, kOffPhiLo = 4 * kAtom;
+constexpr uint32_t kOffOHi = 0, kOffOLo = 2 * kAtom, kOffWHi = 4 * kAtom, kOffWLo = 6 * kAtom;
+constexpr uint32_t kAColBytes = 64 * 128;         // one column of 32 entries, 64 rows
+constexpr uint32_t kAHalfBytes = 5 * kAColBytes;  // N = 144 needs 5 columns (160 entries)
+constexpr uint32_t kOffAHi = 8 * kAtom, kOffALo = kOffAHi + kAHalfBytes;
+constexpr uint32_t kOffBar = kOffALo + kAHalfBytes;
+enum { kBarFullA, kBarReadyPhi, kBarReadyA, kBarFreeA, kBarAcc1, kBarReadyO, kBarReadyW, kBarFreeR0, kBarAcc2,
+       kNumBars };
+constexpr uint32_t kOffMisc = kOffBar + 8 * kNumBars;
+constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
+constexpr uint32_t kColAcc1 = 0, kColAcc2 = 256;  // D1: 144 columns; D2: 128 columns
+static_assert(kOffAHi % 1024 == 0 && kSmem <= 232448, "apply shared memory");
+}  // namespace appm
 
-// grid (nq, BH), 256 threads.  out: fp32 [BH, N, d].  proj: fp32 [d][d] or null (identity).
-__global__ void __launch_bounds__(256)
-    sla_apply_kernel(const uint16_t *__restrict__ q, const float *__restrict__ sums, const float *__restrict__ proj,
-                     int N, int nq, int phi, float *__restrict__ out)
+// hi keeps the sign, exponent and top 10 mantissa bits (exact in TF32); lo = x - hi exactly.
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+// Writes 4 consecutive K values (chunk c of 8 in a 128-byte row) of row r of a K-major,
+// 128-byte swizzled atom, as hi and lo.
+__device__ __forceinline__ void put_hilo(uint8_t *hi, uint8_t *lo, int r, int c, float4 x)
 {
-    extern __shared__ __align__(16) float sm[];
-    float *pq = sm + kApplyPhi, *st = sm + kApplyState, *den = sm + kApplyDen;
-    const int64_t bh = blockIdx.y;
-    const int i = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint16_t *qh = q + bh * int64_t(N) * kD;
-    for (int r = warp; r < kQBlk; r += 8) {
-        const int64_t tok = int64_t(i) * kQBlk + r;
-        float x[4];
-        load_row4(qh, tok, N, lane, x);
-        if (tok < N) phi_row_warp(x, phi);
-        *reinterpret_cast<float4 *>(pq + r * kApplyLd + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+    const float4 h = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+    const uint32_t off = uint32_t(r) * 128u + (uint32_t(c ^ (r & 7)) << 4);
+    *reinterpret_cast<float4 *>(hi + off) = h;
+    *reinterpret_cast<float4 *>(lo + off) = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+}
+
+// grid (nq, heads), appm::kThreads threads, appm::kSmem bytes.  tm_sums: map of the summed
+// states as rows of 136 floats (row (bh * nq + i) * 128 + a; third dimension 1), box {32, 64}.
+__global__ void __launch_bounds__(appm::kThreads, 1)
+    sla_apply_mma_kernel(const __grid_constant__ CUtensorMap tm_sums, const uint16_t *__restrict__ q,
+                         const float *__restrict__ proj, int N, int nq, int phi, float *__restrict__ out)
+{
+    using namespace appm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x, bh = blockIdx.y;
+    const bool has_proj = proj != nullptr;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    auto bar = [&](int b) -> uint32_t { return sbase + kOffBar + 8u * uint32_t(b); };
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kNumBars; ++b)
+            mbar_init(bar(b), (b == kBarReadyPhi || b == kBarReadyA || b == kBarReadyO || b == kBarReadyW) ? 4 : 1);
+        *abort_flag = 0;
+        fence_barrier_init();
     }
-    const float4 *ssrc = reinterpret_cast<const float4 *>(sums + (bh * nq + i) * int64_t(kStateFloats));
-    for (int e = tid; e < kStateFloats / 4; e += 256) reinterpret_cast<float4 *>(st)[e] = __ldg(ssrc + e);
+    if (warp == kWarpIssue) tmem_alloc(sbase + kOffMisc, 512);
+    tc_fence_before();
     __syncthreads();
-    // normaliser of each row: phi(q_r) . z_i (column 128 of the state), one warp per row
-    for (int r = warp; r < kQBlk; r += 8) {
-        float s = 0.0f;
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int64_t arow = (int64_t(bh) * nq + i) * 128;  // first row of A_i in the summed states
+
+    if (warp == kWarpIssue) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_sums);
+            bool ok = true;
+            int loads = 0;  // A halves issued
+            const uint32_t id1 = idesc_tf32_f32(128, 144, false, true), id2 = idesc_tf32_f32(128, 128, false, false);
+            for (int h = 0; h < 2 && ok; ++h) {
+                if (h == 1) ok = mbar_wait(bar(kBarFreeA), 0, abort_flag);  // half 0's MMAs done
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar(kBarFullA), kAHalfBytes);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s = fmaf(pq[r * kApplyLd + 4 * lane + e], st[(4 * lane + e) * kStateCols + kD], s);
+                for (int c = 0; c < 5; ++c)
+                    tma_load_3d(sbase + kOffAHi + uint32_t(c) * kAColBytes, &tm_sums, bar(kBarFullA), 32 * c,
+                                int(arow + 64 * h), 0);
+                ++loads;
+                ok = (h > 0 || mbar_wait(bar(kBarReadyPhi), 0, abort_flag)) && mbar_wait(bar(kBarReadyA), h, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == 0) den[r] = s;
-    }
-    // numerator: rows r = ty + 16 m (m < 8), columns 8 tx .. 8 tx + 7
-    const int ty = tid >> 4, tx = tid & 15;
-    float acc[8][8];
+                for (int kk = 0; kk < 8; ++kk) {
+                    // phi: K-atom 2h + kk/4, 32 bytes per step; A_i: 8 rows (two 4-row atoms)
+                    const uint32_t pa = uint32_t(2 * h + kk / 4) * kAtom + 32u * uint32_t(kk & 3);
+                    const uint64_t ahi = sdesc(sbase + kOffPhiHi + pa, 1024, SWZ_128B);
+                    const uint64_t alo = sdesc(sbase + kOffPhiLo + pa, 1024, SWZ_128B);
+                    const uint64_t bhi = sdesc_mn32(sbase + kOffAHi + 1024u * kk, kAColBytes, 512);
+                    const uint64_t blo = sdesc_mn32(sbase + kOffALo + 1024u * kk, kAColBytes, 512);
+                    mma_tf32(tmem + kColAcc1, ahi, bhi, id1, (h | kk) != 0);
+                    mma_tf32(tmem + kColAcc1, ahi, blo, id1, 1);
+                    mma_tf32(tmem + kColAcc1, alo, bhi, id1, 1);
+                }
+                tc_commit(bar(h == 0 ? kBarFreeA : kBarAcc1));
+            }
+            for (int h = 0; h < 2 && ok && has_proj; ++h) {
+                ok = mbar_wait(bar(kBarReadyO), h, abort_flag) && mbar_wait(bar(kBarReadyW), h, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[m][c] = 0.0f;
-    for (int a = 0; a < kD; a += 4) {
-        float4 p[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) p[m] = *reinterpret_cast<const float4 *>(pq + (ty + 16 * m) * kApplyLd + a);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float4 s0 = *reinterpret_cast<const float4 *>(st + (a + e) * kStateCols + 8 * tx);
-            const float4 s1 = *reinterpret_cast<const float4 *>(st + (a + e) * kStateCols + 8 * tx + 4);
-            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const float pm = e == 0 ? p[m].x : e == 1 ? p[m].y : e == 2 ? p[m].z : p[m].w;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) acc[m][c] = fmaf(pm, sv[c], acc[m][c]);
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t pa = uint32_t(kk / 4) * kAtom + 32u * uint32_t(kk & 3);
+                    const uint64_t ahi = sdesc(sbase + kOffOHi + pa, 1024, SWZ_128B);
+                    const uint64_t alo = sdesc(sbase + kOffOLo + pa, 1024, SWZ_128B);
+                    const uint64_t bhi = sdesc(sbase + kOffWHi + pa, 1024, SWZ_128B);
+                    const uint64_t blo = sdesc(sbase + kOffWLo + pa, 1024, SWZ_128B);
+                    mma_tf32(tmem + kColAcc2, ahi, bhi, id2, (h | kk) != 0);
+                    mma_tf32(tmem + kColAcc2, ahi, blo, id2, 1);
+                    mma_tf32(tmem + kColAcc2, alo, bhi, id2, 1);
+                }
+                tc_commit(bar(h == 0 ? kBarFreeR0 : kBarAcc2));
+            }
+            // the loads and MMAs issued have completed before the CTA's memory is released
+            bool drained = loads == 0 || drain_wait(bar(kBarFullA), uint32_t(loads - 1) & 1u);
+            if (ok) drained = drain_wait(bar(has_proj ? kBarAcc2 : kBarAcc1), 0) && drained;
+            if (!ok || !drained) {
+                *abort_flag = 1;
+                atomicExch(&g_sla_status, 6);
             }
         }
-    }
-    __syncthreads();  // phi(Q) and the state are consumed
-    // O_lin = numerator / normaliser (0 for a row without marginal keys) into the state
-    // region; W^T into the phi(Q) region
-    float *ol = st, *wt = pq;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int r = ty + 16 * m;
-        const float dn = den[r];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[m][c] = dn > 0.0f ? __fdiv_rn(acc[m][c], dn) : 0.0f;
-        *reinterpret_cast<float4 *>(ol + r * kApplyLd + 8 * tx) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-        *reinterpret_cast<float4 *>(ol + r * kApplyLd + 8 * tx + 4) =
-            make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
-    }
-    if (proj) {
-        for (int e = tid; e < kD * kD; e += 256) {
-            const int c = e / kD, f = e % kD;  // W[c][f] -> W^T[f][c]
-            wt[f * kApplyLd + c] = __ldg(proj + e);
+    } else if (warp >= 4) {
+        // ---- operand warps: A_i halves, then W halves
+        const int t = threadIdx.x - 128;
+        bool ok = true;
+        for (int h = 0; h < 2 && ok; ++h) {
+            ok = mbar_wait(bar(kBarFullA), h, abort_flag);
+            if (!ok) break;
+            float4 *ahi = reinterpret_cast<float4 *>(smem + kOffAHi), *alo = reinterpret_cast<float4 *>(smem + kOffALo);
+            for (int e = t; e < int(kAHalfBytes / 16); e += 128) {
+                const float4 x = ahi[e];
+                const float4 hh = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+                ahi[e] = hh;
+                alo[e] = make_float4(x.x - hh.x, x.y - hh.y, x.z - hh.z, x.w - hh.w);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarReadyA));
         }
-        __syncthreads();
-        // out[r][c] = sum_f O_lin[r][f] W[c][f]
+        for (int h = 0; h < 2 && ok && has_proj; ++h) {
+            // R0 is free once GEMM1 (half 0) or the first half of GEMM2 (half 1) is done
+            ok = mbar_wait(bar(h == 0 ? kBarAcc1 : kBarFreeR0), 0, abort_flag);
+            if (!ok) break;
+            // row c = t of W, features 64h .. 64h+63
+            const float4 *wr = reinterpret_cast<const float4 *>(proj + int64_t(t) * kD + 64 * h);
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
+            for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) acc[m][c] = 0.0f;
-        for (int f = 0; f < kD; f += 4) {
-            float4 o4[8];
+                for (int c = 0; c < 8; ++c)
+                    put_hilo(smem + kOffWHi + a * kAtom, smem + kOffWLo + a * kAtom, t, c, __ldg(wr + 8 * a + c));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarReadyW));
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicExch(&g_sla_status, 6);
+        }
+    } else {
+        // ---- row warps: thread r = row r of the query block.  The row of q stays packed
+        // (bf16 pairs) in registers; values are unpacked 4 features (one 16-byte chunk of the
+        // phi tile) at a time.
+        const int r = threadIdx.x;
+        const int64_t tok = int64_t(i) * kQBlk + r;
+        uint4 qp[kD / 8];
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(q + (int64_t(bh) * N + (tok < N ? tok : 0)) * kD);
 #pragma unroll
-            for (int m = 0; m < 8; ++m) o4[m] = *reinterpret_cast<const float4 *>(ol + (ty + 16 * m) * kApplyLd + f);
+            for (int u = 0; u < kD / 8; ++u) qp[u] = tok < N ? __ldg(src + u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        auto unpack4 = [&](int c4) -> float4 {  // features 4 c4 .. 4 c4 + 3
+            const uint4 &w = qp[c4 >> 1];
+            const uint32_t lo = (c4 & 1) ? w.z : w.x, hi = (c4 & 1) ? w.w : w.y;
+            return make_float4(__uint_as_float(lo << 16), __uint_as_float(lo & 0xFFFF0000u),
+                               __uint_as_float(hi << 16), __uint_as_float(hi & 0xFFFF0000u));
+        };
+        // phi = softmax over the features: exp(x - max) / sum.  The 1/sum factor multiplies
+        // the numerator and the normaliser of O_lin alike, so it is not applied here (the
+        // ratio is the same); elu + 1 has no such factor.
+        float m = 0.0f;
+        if (phi == 0) {
+            m = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float4 w0 = *reinterpret_cast<const float4 *>(wt + (f + e) * kApplyLd + 8 * tx);
-                const float4 w1 = *reinterpret_cast<const float4 *>(wt + (f + e) * kApplyLd + 8 * tx + 4);
-                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            for (int c4 = 0; c4 < kD / 4; ++c4) {
+                const float4 x = unpack4(c4);
+                m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
+            }
+        }
+        auto phi1 = [&](float v) -> float { return phi == 0 ? expf(v - m) : (v > 0.0f ? v + 1.0f : expf(v)); };
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const float om = e == 0 ? o4[m].x : e == 1 ? o4[m].y : e == 2 ? o4[m].z : o4[m].w;
+        for (int c4 = 0; c4 < kD / 4; ++c4) {
+            float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (tok < N) {
+                x = unpack4(c4);
+                x = make_float4(phi1(x.x), phi1(x.y), phi1(x.z), phi1(x.w));
+            }
+            put_hilo(smem + kOffPhiHi + (c4 >> 3) * kAtom, smem + kOffPhiLo + (c4 >> 3) * kAtom, r, c4 & 7, x);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarReadyPhi));
+        // O_lin = D1 / normaliser
+        bool ok = mbar_wait(bar(kBarAcc1), 0, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        const uint32_t lrow = uint32_t(32 * warp) << 16;
+        float4 *o = reinterpret_cast<float4 *>(out + (int64_t(bh) * N + tok) * kD);
+        if (ok) {
+            tc_fence_after();
+            uint32_t dn;
+            tmem_ld1_wait(tmem + lrow + kColAcc1 + 128, dn);
+            const float den = __uint_as_float(dn);
+            const float rden = den > 0.0f ? __frcp_rn(den) : 0.0f;  // 0: no marginal key, O_lin = 0
+            // 32 columns of O_lin (chunk cb) -> hi/lo O tile (GEMM2) or the output
+            for (int cb = 0; cb < 4; ++cb) {
+                if (has_proj && (cb & 1) == 0) {
+                    // a K half of GEMM2 starts: its O tiles reuse R0 once the MMAs before are done
+                    if (cb == 2) ok = mbar_wait(bar(kBarFreeR0), 0, abort_flag);
+                    if (!ok) break;
+                }
+                uint32_t v[32];
+                tmem_ld32_wait(tmem + lrow + kColAcc1 + 32 * cb, v);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[m][c] = fmaf(om, wv[c], acc[m][c]);
+                for (int c = 0; c < 8; ++c) {
+                    const float4 x = make_float4(__uint_as_float(v[4 * c]) * rden, __uint_as_float(v[4 * c + 1]) * rden,
+                                                 __uint_as_float(v[4 * c + 2]) * rden,
+                                                 __uint_as_float(v[4 * c + 3]) * rden);
+                    if (has_proj)
+                        put_hilo(smem + kOffOHi + (cb & 1) * kAtom, smem + kOffOLo + (cb & 1) * kAtom, r, c, x);
+                    else if (tok < N)
+                        o[8 * cb + c] = x;
+                }
+                if (has_proj && (cb & 1) == 1) {
+                    tc_fence_before();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(kBarReadyO));
+                }
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok && has_proj) {
+                ok = __all_sync(0xffffffffu, mbar_wait(bar(kBarAcc2), 0, abort_flag));
+                if (ok) {
+                    tc_fence_after();
+                    for (int cb = 0; cb < 4; ++cb) {
+                        uint32_t v[32];
+                        tmem_ld32_wait(tmem + lrow + kColAcc2 + 32 * cb, v);
+                        if (tok < N) {
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                o[8 * cb + c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]),
+                                                            __uint_as_float(v[4 * c + 2]), __uint_as_float(v[4 * c + 3]));
+                        }
+                    }
                 }
             }
         }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            atomicExch(&g_sla_status, 6);
+        }
     }
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-        const int64_t tok = int64_t(i) * kQBlk + ty + 16 * m;
-        if (tok >= N) continue;
-        float *o = out + (bh * N + tok) * kD + 8 * tx;
-        *reinterpret_cast<float4 *>(o) = make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-        *reinterpret_cast<float4 *>(o + 4) = make_float4(acc[m][4], acc[m][5], acc[m][6], acc[m][7]);
-    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == kWarpIssue) tmem_dealloc(tmem, 512);
 }
 
 __global__ void sla_critical_kernel(const uint8_t *__restrict__ classes, int64_t n, uint8_t *__restrict__ keep)
@@ -499,8 +670,8 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
                                       int(state_smem))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_sum_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(summ::kSmem))) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(sla_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(kApplySmemBytes))) != cudaSuccess)
+            (e = cudaFuncSetAttribute(sla_apply_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(appm::kSmem))) != cudaSuccess)
             return e;
         attr_set[dev] = true;
     }
@@ -534,8 +705,13 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
         sla_sum_mma_kernel<<<dim3(unsigned((nq + nt - 1) / nt), unsigned(kStateFloats / summ::kM), unsigned(g)),
                              summ::kThreads, summ::kSmem, st>>>(tm_state, tm_c, nq, nk, nt, sums);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        sla_apply_kernel<<<dim3(unsigned(nq), unsigned(g)), 256, kApplySmemBytes, st>>>(
-            static_cast<const uint16_t *>(q) + h0 * tok, sums, proj, N, nq, phi, out + h0 * tok);
+        CUtensorMap tm_sums;
+        const uint64_t srows = uint64_t(g) * uint64_t(nq) * kD;
+        if (!encode_tmap_3d_f32(&tm_sums, sums, kStateCols, srows, 1, kStateCols * sizeof(float),
+                                srows * kStateCols * sizeof(float), 32, 64, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
+            return cudaErrorInvalidValue;
+        sla_apply_mma_kernel<<<dim3(unsigned(nq), unsigned(g)), appm::kThreads, appm::kSmem, st>>>(
+            tm_sums, static_cast<const uint16_t *>(q) + h0 * tok, proj, N, nq, phi, out + h0 * tok);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
