@@ -8,6 +8,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <numeric>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -174,10 +176,46 @@ static sa_status get_workspace(WsLock &lock, size_t bytes, uint8_t **out)
     return SA_OK;
 }
 
+// Page-locked host staging for small tables that a call uploads (variable-length
+// batches), per device, grow-only.  Used with the workspace lock held; the event marks the
+// last upload, which must have left the buffer before it is overwritten.
+struct HostStage {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+    cudaEvent_t ev = nullptr;
+};
+static HostStage g_stage[64];
+
+static sa_status upload_table(const void *src, size_t n, void *dst, cudaStream_t st)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SA_ERR_CUDA;
+    HostStage &h = g_stage[dev];
+    if (!h.ev) {
+        if (cudaEventCreateWithFlags(&h.ev, cudaEventDisableTiming) != cudaSuccess) return SA_ERR_CUDA;
+    } else if (cudaEventSynchronize(h.ev) != cudaSuccess) {
+        return SA_ERR_CUDA;
+    }
+    if (h.bytes < n) {
+        if (h.ptr) cudaFreeHost(h.ptr);
+        h.ptr = nullptr;
+        h.bytes = 0;
+        if (cudaMallocHost(&h.ptr, n) != cudaSuccess) {
+            cudaGetLastError();
+            return SA_ERR_OOM;
+        }
+        h.bytes = n;
+    }
+    std::memcpy(h.ptr, src, n);
+    if (cudaMemcpyAsync(dst, h.ptr, n, cudaMemcpyHostToDevice, st) != cudaSuccess) return SA_ERR_CUDA;
+    return cudaEventRecord(h.ev, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
 static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t *k8,
                                 const float *sk, const uint8_t *v8, const float *sv, void *o,
                                 const Shape &s, float sm_scale, const uint8_t *mask,
-                                cudaStream_t st, bool causal = false, const float *addend = nullptr)
+                                cudaStream_t st, bool causal = false, const float *addend = nullptr,
+                                const SeqTable &seq = SeqTable())
 {
     AttnArgs a;
     const uint64_t rows = uint64_t(s.BH() * s.Npad());
@@ -199,13 +237,15 @@ static sa_status attention_core(const int8_t *q8, const float *sq, const int8_t 
     a.sm_scale = sm_scale;
     a.causal = causal ? 1 : 0;
     a.addend = addend;
+    a.seq = seq;
     return launch_attention(a, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
 // Prologue into the library workspace, then the fused attention kernel (validated args).
 static sa_status attn_fwd_device(const void *q, const void *k, const void *v, void *o,
                                  const Shape &s, float sm_scale, const uint8_t *block_mask,
-                                 cudaStream_t st, bool causal = false, const float *addend = nullptr)
+                                 cudaStream_t st, bool causal = false, const float *addend = nullptr,
+                                 const SeqTable &seq = SeqTable())
 {
     const WsLayout L = ws_layout(s);
     WsLock lock;
@@ -219,12 +259,12 @@ static sa_status attn_fwd_device(const void *q, const void *k, const void *v, vo
     float *sk = reinterpret_cast<float *>(ws + L.sk);
     float *sv = reinterpret_cast<float *>(ws + L.sv);
     if (launch_quantize_qk(q, k, s, q8, sq, k8, sk, reinterpret_cast<float *>(ws + L.kmean),
-                           reinterpret_cast<double *>(ws + L.kpart), st) != cudaSuccess)
+                           reinterpret_cast<double *>(ws + L.kpart), st, seq) != cudaSuccess)
         return SA_ERR_CUDA;
-    if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st) !=
+    if (launch_quantize_v(v, s, v8, sv, reinterpret_cast<uint32_t *>(ws + L.vamax), st, seq) !=
         cudaSuccess)
         return SA_ERR_CUDA;
-    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st, causal, addend);
+    return attention_core(q8, sq, k8, sk, v8, sv, o, s, sm_scale, block_mask, st, causal, addend, seq);
 }
 
 // ------------------------------------------------------------------ host-buffer pipeline
@@ -683,31 +723,70 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     sa_status r = check_ptrs({q, k, v, o});
     if (r != SA_OK) return r;
-    // validate every sequence and size the workspace for the largest before any launch
-    size_t need = 0;
+    // every sequence is valid on its own; start[i] = its first token in the packed batch
+    std::vector<int64_t> start(static_cast<size_t>(nseq) + 1, 0);
     for (int i = 0; i < nseq; ++i) {
         Shape s;
         if ((r = check_shape(1, H, seqlens[i], d, &s)) != SA_OK) return r;
+        start[i + 1] = start[i] + seqlens[i];
+    }
+    if (start[nseq] > INT_MAX / 8 || int64_t(H) * start[nseq] > INT64_MAX / kD) return SA_ERR_INVALID_ARG;
+    // Groups: sequences taken longest first; a group runs as one prologue and one attention
+    // launch over heads padded to its longest sequence, and takes the next sequence while
+    // the padded size stays within twice the group's own (or below 2^20 padded
+    // token-heads, where the padding costs little).
+    std::vector<int> ord(static_cast<size_t>(nseq));
+    std::iota(ord.begin(), ord.end(), 0);
+    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return seqlens[a] > seqlens[b]; });
+    struct Group {
+        int first, count;
+        int64_t nmax;
+    };
+    std::vector<Group> groups;
+    size_t need = 0;
+    for (int g0 = 0; g0 < nseq;) {
+        const int64_t nmax = seqlens[ord[g0]], pmax = padded_len(nmax);
+        int64_t own = pmax;
+        int cnt = 1;
+        while (g0 + cnt < nseq) {
+            const int64_t own2 = own + padded_len(seqlens[ord[g0 + cnt]]), pad2 = int64_t(cnt + 1) * pmax;
+            if (pad2 > 2 * own2 && pad2 * H > (int64_t(1) << 20)) break;
+            own = own2;
+            ++cnt;
+        }
+        Shape s;
+        if ((r = check_shape(cnt, H, int(nmax), d, &s)) != SA_OK) return r;
         need = std::max(need, align256(ws_layout(s).total));
+        groups.push_back({g0, cnt, nmax});
+        g0 += cnt;
+    }
+    // device table after the largest group's workspace: the lengths in group order, then
+    // the first row (of d elements) of every head in q, k, v and o
+    const size_t lb = align256(size_t(nseq) * sizeof(int)), tb = lb + size_t(nseq) * H * sizeof(int64_t);
+    std::vector<uint8_t> table(tb, 0);
+    int *lens = reinterpret_cast<int *>(table.data());
+    int64_t *rows = reinterpret_cast<int64_t *>(table.data() + lb);
+    for (int i = 0; i < nseq; ++i) {
+        const int sq = ord[i];
+        lens[i] = seqlens[sq];
+        for (int h = 0; h < H; ++h) rows[size_t(i) * H + h] = int64_t(H) * start[sq] + int64_t(h) * seqlens[sq];
     }
     if ((r = check_device()) != SA_OK) return r;
     WsLock lock;
     uint8_t *ws = nullptr;
-    if ((r = get_workspace(lock, need, &ws)) != SA_OK) return r;
+    if ((r = get_workspace(lock, need + tb, &ws)) != SA_OK) return r;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // sequence i occupies H * N_i * d consecutive elements of each tensor, after those of
-    // the sequences before it; each is an independent [1, H, N_i, d] problem
-    int64_t off = 0;
-    for (int i = 0; i < nseq; ++i) {
+    if ((r = upload_table(table.data(), tb, ws + need, st)) != SA_OK) return r;
+    const int *dlens = reinterpret_cast<const int *>(ws + need);
+    const int64_t *drows = reinterpret_cast<const int64_t *>(ws + need + lb);
+    for (const Group &g : groups) {
         Shape s;
-        check_shape(1, H, seqlens[i], d, &s);
-        const auto *qi = static_cast<const uint16_t *>(q) + off, *ki = static_cast<const uint16_t *>(k) + off,
-                   *vi = static_cast<const uint16_t *>(v) + off;
-        auto *oi = static_cast<uint16_t *>(o) + off;
-        if ((reinterpret_cast<uintptr_t>(qi) & 15u) != 0) return SA_ERR_MISALIGNED;
-        r = attn_fwd_device(qi, ki, vi, oi, s, sm_scale, nullptr, st, causal != 0);
-        if (r != SA_OK) return r;
-        off += int64_t(H) * seqlens[i] * kD;
+        check_shape(g.count, H, int(g.nmax), d, &s);
+        SeqTable t;
+        t.len = dlens + g.first;
+        t.row = drows + size_t(g.first) * H;
+        t.H = H;
+        if ((r = attn_fwd_device(q, k, v, o, s, sm_scale, nullptr, st, causal != 0, nullptr, t)) != SA_OK) return r;
     }
     return SA_OK;
 }
@@ -793,6 +872,13 @@ sa_status sa_release_workspace(void)
         cudaFree(w.ptr);
         w.ptr = nullptr;
         w.bytes = 0;
+    }
+    HostStage &h = g_stage[dev];
+    if (h.ptr) {
+        if (cudaEventSynchronize(h.ev) != cudaSuccess) return SA_ERR_CUDA;
+        cudaFreeHost(h.ptr);
+        h.ptr = nullptr;
+        h.bytes = 0;
     }
     return SA_OK;
 }

@@ -671,9 +671,11 @@ static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(attn_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(pairs::kSmemAlloc));
-        if (e != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(attn_pairs_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(pairs::kSmemAlloc))) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(attn_pairs_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(pairs::kSmemAlloc))) != cudaSuccess)
+            return e;
         attr_set[dev] = true;
     }
     int sms = 0;
@@ -681,9 +683,14 @@ static cudaError_t launch_attention_pairs(const AttnArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const int npairs = a.BH * ((a.nq + 1) / 2);
     const int grid = npairs < sms ? npairs : sms;
-    attn_pairs_kernel<<<grid, pairs::kThreads, pairs::kSmemAlloc, st>>>(
-        a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale, a.v_scale, a.o, a.BH, a.N, a.Npad, a.nq, a.nk,
-        a.sm_scale, a.causal);
+    if (a.seq.len)
+        attn_pairs_kernel<true><<<grid, pairs::kThreads, pairs::kSmemAlloc, st>>>(
+            a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale, a.v_scale, a.o, a.BH, a.N, a.Npad, a.nq, a.nk,
+            a.sm_scale, a.causal, a.seq);
+    else
+        attn_pairs_kernel<false><<<grid, pairs::kThreads, pairs::kSmemAlloc, st>>>(
+            a.tm_q, a.tm_k, a.tm_v, a.q_scale, a.k_scale, a.v_scale, a.o, a.BH, a.N, a.Npad, a.nq, a.nk,
+            a.sm_scale, a.causal, a.seq);
     return cudaGetLastError();
 }
 

@@ -182,12 +182,17 @@ __device__ __forceinline__ void p_row(const uint32_t (&s0)[32], const uint32_t (
 
 }  // namespace pairs
 
+// VARLEN: head bh has seq_tokens(seq, bh, N) tokens and its output rows start at
+// seq_row0(seq, bh, N); N, Npad, nq and nk are those of the longest head (the strides of the
+// quantised buffers and scales), and the pairs past a head's own tiles are skipped by every
+// role alike.
+template <bool VARLEN>
 __global__ void __launch_bounds__(pairs::kThreads, 1)
     attn_pairs_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ q_scale,
                       const float *__restrict__ k_scale, const float *__restrict__ v_scale,
                       __nv_bfloat16 *__restrict__ out, int BH, int N, int Npad, int nq, int nk,
-                      float sm_scale, int causal)
+                      float sm_scale, int causal, SeqTable seq)
 {
     using pairs::kStages;
     using pairs::kThreads;
@@ -267,12 +272,21 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
     const uint32_t tmem = *tmem_base_slot;
 
     const int npairs_h = (nq + 1) / 2, npairs = BH * npairs_h;
-    const int nsteps = (nk + 1) / 2;  // every block kept: blocks 2j and 2j+1 form step j
-    const bool odd_tail = (nk & 1) != 0;  // the last step then has one block
+    // the tokens, query tiles and key steps of head bh (every block kept: blocks 2j and
+    // 2j+1 form step j; with an odd block count the last step has one block)
+    struct Geo {
+        int n, nq, nk, nsteps;
+        bool odd;
+    };
+    auto geo = [&](int bh) -> Geo {
+        if (!VARLEN) return Geo{N, nq, nk, (nk + 1) / 2, (nk & 1) != 0};
+        const int n = seq_tokens(seq, bh, N), q = (n + 127) / 128, k = (n + 63) / 64;
+        return Geo{n, q, k, (k + 1) / 2, (k & 1) != 0};
+    };
     // causal: the pair (qa, qa + 1) needs the steps up to tile qa + 1's diagonal, qa + 2 of
     // them (qa + 1 for a lone last tile); tile qa's last step is then fully masked
-    auto pair_steps = [&](int qa) -> int {
-        return causal ? min(nsteps, qa + (qa + 1 < nq ? 2 : 1)) : nsteps;
+    auto pair_steps = [&](int qa, const Geo &g) -> int {
+        return causal ? min(g.nsteps, qa + (qa + 1 < g.nq ? 2 : 1)) : g.nsteps;
     };
     // The work items of this CTA, the same sequence for every role: item r*G + b of round r
     // (G CTAs, b = this CTA).  Without causality every pair costs the same, and pairs go in
@@ -298,9 +312,11 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             // preference to the Q tiles, which one CTA reads once (DRAM traffic per launch at
             // 40 x 75600: 2.43 GB with the hints, 2.49 GB without; 1.94 GB algorithmic)
             const uint64_t pol_kv = l2_policy_evict_last(), pol_q = l2_policy_evict_first();
-            for (int r = 0, p = item(0); p < npairs; p = item(++r), ++pl) {
+            for (int r = 0, p = item(0); p < npairs; p = item(++r)) {
                 const int bh = pair_head(p), qa = pair_qa(p);
-                const bool hasb = qa + 1 < nq;
+                const Geo ge = geo(bh);
+                if (VARLEN && qa >= ge.nq) continue;
+                const bool hasb = qa + 1 < ge.nq;
                 if (pl >= 1 && ok) ok = mbar_wait(bar(kBarQEmpty), (pl - 1) & 1, abort_flag);
                 if (ok) {
                     mbar_arrive_expect_tx(bar(kBarQFull), (hasb ? 2u : 1u) * kQTileBytes);
@@ -309,10 +325,10 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                         tma_load_2d_hint(sbase + kOffQ + kQTileBytes, &tm_q, bar(kBarQFull), 0,
                                          bh * Npad + qa * 128 + 128, pol_q);
                 }
-                const int ns = pair_steps(qa);
+                const int ns = pair_steps(qa, ge);
                 for (int j = 0; j < ns && ok; ++j, ++g) {
                     const uint32_t st = g % kStages;
-                    const bool two = !(odd_tail && j == nsteps - 1);
+                    const bool two = !(ge.odd && j == ge.nsteps - 1);
                     if (g >= kStages) ok = mbar_wait(bar(kBarKvEmpty + st), ((g / kStages) - 1) & 1, abort_flag);
                     if (!ok) break;
                     const uint32_t kb = sbase + kOffK + st * kKTileBytes;
@@ -327,6 +343,7 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                                          pol_kv);
                     }
                 }
+                ++pl;
             }
             if (!ok) { *abort_flag = 1; record_timeout(); }
         } else if (warp == kWarpMmaQK && lane == 0) {
@@ -334,12 +351,14 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             // S_A(j), S_B(j), S_A(j+1), ... through the one S buffer
             bool ok = true;
             uint32_t g = 0, u = 0, pl = 0;
-            for (int r = 0, p = item(0); p < npairs && ok; p = item(++r), ++pl) {
+            for (int r = 0, p = item(0); p < npairs && ok; p = item(++r)) {
                 const int qa = pair_qa(p);
-                const int ntile = qa + 1 < nq ? 2 : 1;
+                const Geo ge = geo(pair_head(p));
+                if (VARLEN && qa >= ge.nq) continue;
+                const int ntile = qa + 1 < ge.nq ? 2 : 1;
                 ok = mbar_wait(bar(kBarQFull), pl & 1, abort_flag);
                 tc_fence_after();
-                const int ns = pair_steps(qa);
+                const int ns = pair_steps(qa, ge);
                 for (int j = 0; j < ns && ok; ++j, ++g) {
                     const uint32_t st = g % kStages;
                     ok = mbar_wait(bar(kBarKvFull + st), (g / kStages) & 1, abort_flag);
@@ -357,6 +376,7 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                     }
                 }
                 if (ok) tc_commit(bar(kBarQEmpty));
+                ++pl;
             }
             if (!ok) { *abort_flag = 1; record_timeout(); }
         } else if (warp == kWarpMmaPV && lane == 0) {
@@ -365,11 +385,13 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             uint32_t g = 0, c[2] = {0, 0}, o[2] = {0, 0};
             for (int r = 0, p = item(0); p < npairs && ok; p = item(++r)) {
                 const int qa = pair_qa(p);
-                const int ntile = qa + 1 < nq ? 2 : 1;
-                const int ns = pair_steps(qa);
+                const Geo ge = geo(pair_head(p));
+                if (VARLEN && qa >= ge.nq) continue;
+                const int ntile = qa + 1 < ge.nq ? 2 : 1;
+                const int ns = pair_steps(qa, ge);
                 for (int j = 0; j < ns && ok; ++j, ++g) {
                     const uint32_t st = g % kStages;
-                    const int nkk = (odd_tail && j == nsteps - 1) ? 2 : 4;  // K = 64 or 128 keys
+                    const int nkk = (ge.odd && j == ge.nsteps - 1) ? 2 : 4;  // K = 64 or 128 keys
                     ok = mbar_wait(bar(kBarKvFull + st), (g / kStages) & 1, abort_flag);
                     const uint32_t vb = sbase + kOffV + st * 2 * kVHalfBytes;
                     for (int t = 0; t < ntile && ok; ++t) {
@@ -410,16 +432,17 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
         uint32_t c = 0, o = 0;  // steps and tiles this warpgroup has processed
         for (int r = 0, p = item(0); p < npairs; p = item(++r)) {
             const int bh = pair_head(p), qt = pair_qa(p) + t;
-            if (qt >= nq) continue;  // tile B of the last pair of an odd tile count
+            const Geo ge = geo(bh);
+            if (qt >= ge.nq) continue;  // tile B of the last pair of an odd tile count (or past the head)
             const int qrow = qt * 128 + row;
             const float sq = q_scale[int64_t(bh) * nq + qt];
             const float *ksrow = k_scale + int64_t(bh) * nk;
             float m = -INFINITY;
-            const int ns = pair_steps(qt - t);
+            const int ns = pair_steps(qt - t, ge);
             for (int j = 0; j < ns; ++j, ++c) {
-                const bool two = !(odd_tail && j == nsteps - 1);
+                const bool two = !(ge.odd && j == ge.nsteps - 1);
                 const float ks0 = ksrow[2 * j], ks1 = two ? ksrow[2 * j + 1] : 0.0f;
-                int nv0 = min(64, N - 128 * j), nv1 = two ? min(64, N - 128 * j - 64) : 0;
+                int nv0 = min(64, ge.n - 128 * j), nv1 = two ? min(64, ge.n - 128 * j - 64) : 0;
                 if (causal) {
                     // this row keeps the keys up to itself
                     nv0 = max(0, min(nv0, qrow - 128 * j + 1));
@@ -527,12 +550,12 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
                 const float l = __uint_as_float(lbits);
                 const float inv_l = l > 0.0f ? __frcp_rn(l) : 0.0f;
                 const float *svp = v_scale + int64_t(bh) * kD;
-                __nv_bfloat16 *orow = out + (int64_t(bh) * N + qrow) * kD;
+                __nv_bfloat16 *orow = out + ((VARLEN ? seq_row0(seq, bh, N) : int64_t(bh) * N) + qrow) * kD;
 #pragma unroll 1
                 for (int h = 0; h < 4; ++h) {
                     uint32_t ov[32];
                     tmem_ld32_wait(oa + 32 * h, ov);
-                    if (qrow < N) {
+                    if (qrow < ge.n) {
 #pragma unroll
                         for (int cidx = 0; cidx < 4; ++cidx) {
                             uint32_t w[4];

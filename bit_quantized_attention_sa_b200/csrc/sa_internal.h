@@ -26,12 +26,32 @@ struct Shape {
     int64_t nchunks() const { return cdiv(N, kMeanChunk); }
 };
 
+// Packed variable-length batches: head bh = b * H + h holds len[b] tokens, whose rows (d
+// elements each) start at row[bh] in q, k, v and o; the quantised buffers, scales and
+// partial sums keep the uniform layout of a Shape whose N is the longest sequence.  With
+// len == nullptr every head has Shape::N tokens at row bh * N.
+struct SeqTable {
+    const int *len = nullptr;
+    const int64_t *row = nullptr;
+    int H = 1;
+};
+__device__ __forceinline__ int seq_tokens(const SeqTable &t, int64_t bh, int N)
+{
+    return t.len ? __ldg(t.len + bh / t.H) : N;
+}
+__device__ __forceinline__ int64_t seq_row0(const SeqTable &t, int64_t bh, int N)
+{
+    return t.len ? __ldg(t.row + bh) : bh * int64_t(N);
+}
+
 // ---- prologue (sa_prologue.cu)
 cudaError_t launch_quantize_qk(const void *q, const void *k, const Shape &s, int8_t *q_i8,
                                float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
-                               double *k_partial /* [BH, nchunks, d] */, cudaStream_t st);
+                               double *k_partial /* [BH, nchunks, d] */, cudaStream_t st,
+                               const SeqTable &seq = SeqTable());
 cudaError_t launch_quantize_v(const void *v, const Shape &s, uint8_t *v_t, float *v_scale,
-                              uint32_t *v_amax_bits /* [BH, d] */, cudaStream_t st);
+                              uint32_t *v_amax_bits /* [BH, d] */, cudaStream_t st,
+                              const SeqTable &seq = SeqTable());
 // d = 64 calls: [rows][64] bf16 -> [rows][128] with zero upper channels, and back.
 cudaError_t launch_pad_heads(const void *src, int64_t rows, void *dst, cudaStream_t st);
 cudaError_t launch_unpad_heads(const void *src, int64_t rows, void *dst, cudaStream_t st);
@@ -50,6 +70,7 @@ struct AttnArgs {
     int causal = 0;  // row r keeps only the keys t <= r (mask must then be set)
     // fp32 [B,H,N,d] added to O before its single rounding to bf16 (masked calls), or null
     const float *addend = nullptr;
+    SeqTable seq;  // variable-length heads (unmasked calls only)
 };
 cudaError_t launch_attention(const AttnArgs &a, cudaStream_t st);
 cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k, int BH,

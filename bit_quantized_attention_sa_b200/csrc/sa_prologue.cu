@@ -38,16 +38,18 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&x)[8])
 
 // ---- K channel sums: per (head, 1024-token chunk) fp64 partial sums, fixed order.
 __global__ void __launch_bounds__(kThreads) k_partial_kernel(const uint16_t *__restrict__ k,
-                                                             int N, int nchunks,
-                                                             double *__restrict__ part)
+                                                             int Nmax, int nchunks,
+                                                             double *__restrict__ part, SeqTable seq)
 {
     __shared__ double red[16][kD];
     const int chunk = blockIdx.x;
     const int64_t bh = blockIdx.y;
+    const int N = seq_tokens(seq, bh, Nmax);
     const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
     const int t0 = chunk * kMeanChunk;
+    if (t0 >= N) return;  // past this head's tokens (variable-length batches)
     const int t1 = min(N, t0 + kMeanChunk);
-    const uint16_t *kh = k + bh * int64_t(N) * kD;
+    const uint16_t *kh = k + seq_row0(seq, bh, Nmax) * kD;
     double acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
@@ -69,14 +71,15 @@ __global__ void __launch_bounds__(kThreads) k_partial_kernel(const uint16_t *__r
     }
 }
 
-// mean_k[c] = fp32( (sum over chunks, in order) / N ) in fp64.
-__global__ void __launch_bounds__(kD) k_mean_kernel(const double *__restrict__ part, int N,
-                                                    int nchunks, float *__restrict__ mean)
+// mean_k[c] = fp32( (sum over this head's chunks, in order) / N ) in fp64.
+__global__ void __launch_bounds__(kD) k_mean_kernel(const double *__restrict__ part, int Nmax,
+                                                    int nchunks, float *__restrict__ mean, SeqTable seq)
 {
     const int64_t bh = blockIdx.x;
     const int c = threadIdx.x;
+    const int N = seq_tokens(seq, bh, Nmax), nch = (N + kMeanChunk - 1) / kMeanChunk;
     double s = 0.0;
-    for (int i = 0; i < nchunks; ++i) s += part[(bh * nchunks + i) * kD + c];
+    for (int i = 0; i < nch; ++i) s += part[(bh * nchunks + i) * kD + c];
     mean[bh * kD + c] = float(s / double(N));
 }
 
@@ -162,38 +165,45 @@ __device__ __forceinline__ void quant_block(const uint16_t *__restrict__ src, in
 }
 
 // grid (nq + Npad/64, BH): x < nq quantises Q block x; otherwise K block x - nq
-// (blocks at or past nk only zero-fill the padded key rows).
+// (blocks at or past nk only zero-fill the padded key rows).  With a variable-length
+// table, N is the head's own length and blocks past its padded length are skipped (the
+// attention kernel never reads them); nq, nk and Npad are the strides of the longest.
 __global__ void __launch_bounds__(kThreads, 4)
-    qk_quant_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, int N,
+    qk_quant_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ k, int Nmax,
                     int Npad, int nq, int nk, const float *__restrict__ kmean,
                     int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
-                    int8_t *__restrict__ k_i8, float *__restrict__ k_scale)
+                    int8_t *__restrict__ k_i8, float *__restrict__ k_scale, SeqTable seq)
 {
     __shared__ float red[kThreads / 32];
     const int64_t bh = blockIdx.y;
     const int x = blockIdx.x;
+    const int N = seq_tokens(seq, bh, Nmax), nqh = (N + kQBlk - 1) / kQBlk, nkh = (N + kKBlk - 1) / kKBlk;
+    const int64_t row0 = seq_row0(seq, bh, Nmax);
     if (x < nq) {
-        quant_block<kQBlk>(q + bh * int64_t(N) * kD, N, x * kQBlk, nullptr,
-                           q_i8 + bh * int64_t(Npad) * kD, q_scale + bh * nq + x, red);
+        if (x >= nqh) return;
+        quant_block<kQBlk>(q + row0 * kD, N, x * kQBlk, nullptr, q_i8 + bh * int64_t(Npad) * kD,
+                           q_scale + bh * nq + x, red);
     } else {
         const int j = x - nq;
-        quant_block<kKBlk>(k + bh * int64_t(N) * kD, N, j * kKBlk, kmean + bh * kD,
-                           k_i8 + bh * int64_t(Npad) * kD, j < nk ? k_scale + bh * nk + j : nullptr,
-                           red);
+        if (j * kKBlk >= nqh * kQBlk) return;
+        quant_block<kKBlk>(k + row0 * kD, N, j * kKBlk, kmean + bh * kD, k_i8 + bh * int64_t(Npad) * kD,
+                           j < nkh ? k_scale + bh * nk + j : nullptr, red);
     }
 }
 
 // ---- V: per-channel max |v| (as bf16 magnitude bits; order-free), then codes.
-__global__ void __launch_bounds__(kThreads) v_amax_kernel(const uint16_t *__restrict__ v, int N,
-                                                          uint32_t *__restrict__ amax_bits)
+__global__ void __launch_bounds__(kThreads) v_amax_kernel(const uint16_t *__restrict__ v, int Nmax,
+                                                          uint32_t *__restrict__ amax_bits, SeqTable seq)
 {
     __shared__ uint32_t red[16][kD];
     const int chunk = blockIdx.x;
     const int64_t bh = blockIdx.y;
+    const int N = seq_tokens(seq, bh, Nmax);
     const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
     const int t0 = chunk * kMeanChunk;
+    if (t0 >= N) return;
     const int t1 = min(N, t0 + kMeanChunk);
-    const uint16_t *vh = v + bh * int64_t(N) * kD;
+    const uint16_t *vh = v + seq_row0(seq, bh, Nmax) * kD;
     uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     for (int t = t0 + rs; t < t1; t += 16) {
         const uint4 u = __ldg(reinterpret_cast<const uint4 *>(vh + int64_t(t) * kD + cg * 8));
@@ -222,14 +232,16 @@ __global__ void __launch_bounds__(kThreads) v_amax_kernel(const uint16_t *__rest
 // row c, g = c / 8: the 16 threads of a half-warp, each writing one byte for its own group
 // of 8 channels, then hit 16 different banks, and a thread still reads a whole chunk.
 __global__ void __launch_bounds__(kThreads)
-    v_quant_kernel(const uint16_t *__restrict__ v, int N, int Npad,
+    v_quant_kernel(const uint16_t *__restrict__ v, int Nmax, int Npad,
                    const uint32_t *__restrict__ amax_bits, uint8_t *__restrict__ v_t,
-                   float *__restrict__ v_scale)
+                   float *__restrict__ v_scale, SeqTable seq)
 {
     __shared__ __align__(16) uint8_t tile[kD][kQBlk];
     __shared__ float sv[kD];
     const int64_t bh = blockIdx.y;
     const int t0 = blockIdx.x * kQBlk;
+    const int N = seq_tokens(seq, bh, Nmax);
+    if (blockIdx.x > 0 && t0 >= N) return;  // past this head's padded length (tile 0 writes the scales)
     const int tid = threadIdx.x, cg = tid & 15, rs = tid >> 4;
     if (tid < kD) {
         const float s = __fdiv_rn(bf16_bits_to_f32(amax_bits[bh * kD + tid]), 448.0f);
@@ -237,7 +249,7 @@ __global__ void __launch_bounds__(kThreads)
         if (blockIdx.x == 0) v_scale[bh * kD + tid] = s;
     }
     __syncthreads();
-    const uint16_t *vh = v + bh * int64_t(N) * kD;
+    const uint16_t *vh = v + seq_row0(seq, bh, Nmax) * kD;
     const int swz_chunk = cg & 7, swz_word = cg >> 3;
 #pragma unroll
     for (int i = 0; i < kQBlk * 16 / kThreads; ++i) {
@@ -345,31 +357,31 @@ cudaError_t noalloc_kpart(double **out)
 
 cudaError_t launch_quantize_qk(const void *q, const void *k, const Shape &s, int8_t *q_i8,
                                float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
-                               double *k_partial, cudaStream_t st)
+                               double *k_partial, cudaStream_t st, const SeqTable &seq)
 {
     const int N = int(s.N), Npad = int(s.Npad()), nq = int(s.nq()), nk = int(s.nk());
     const int nch = int(s.nchunks());
     const dim3 g1(nch, unsigned(s.BH()));
-    k_partial_kernel<<<g1, kThreads, 0, st>>>(static_cast<const uint16_t *>(k), N, nch, k_partial);
-    k_mean_kernel<<<unsigned(s.BH()), kD, 0, st>>>(k_partial, N, nch, k_mean);
+    k_partial_kernel<<<g1, kThreads, 0, st>>>(static_cast<const uint16_t *>(k), N, nch, k_partial, seq);
+    k_mean_kernel<<<unsigned(s.BH()), kD, 0, st>>>(k_partial, N, nch, k_mean, seq);
     const dim3 g2(nq + Npad / kKBlk, unsigned(s.BH()));
     qk_quant_kernel<<<g2, kThreads, 0, st>>>(static_cast<const uint16_t *>(q),
                                              static_cast<const uint16_t *>(k), N, Npad, nq, nk,
-                                             k_mean, q_i8, q_scale, k_i8, k_scale);
+                                             k_mean, q_i8, q_scale, k_i8, k_scale, seq);
     return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_v(const void *v, const Shape &s, uint8_t *v_t, float *v_scale,
-                              uint32_t *v_amax_bits, cudaStream_t st)
+                              uint32_t *v_amax_bits, cudaStream_t st, const SeqTable &seq)
 {
     const int N = int(s.N), Npad = int(s.Npad());
     cudaError_t e = cudaMemsetAsync(v_amax_bits, 0, sizeof(uint32_t) * s.BH() * kD, st);
     if (e != cudaSuccess) return e;
     const dim3 g1(unsigned(s.nchunks()), unsigned(s.BH()));
-    v_amax_kernel<<<g1, kThreads, 0, st>>>(static_cast<const uint16_t *>(v), N, v_amax_bits);
+    v_amax_kernel<<<g1, kThreads, 0, st>>>(static_cast<const uint16_t *>(v), N, v_amax_bits, seq);
     const dim3 g2(unsigned(Npad / kQBlk), unsigned(s.BH()));
     v_quant_kernel<<<g2, kThreads, 0, st>>>(static_cast<const uint16_t *>(v), N, Npad, v_amax_bits,
-                                            v_t, v_scale);
+                                            v_t, v_scale, seq);
     return cudaGetLastError();
 }
 

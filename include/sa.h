@@ -143,8 +143,12 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
  * sa_attn_fwd (causal = 0) or sa_attn_fwd_causal without a mask (causal != 0) would compute
  * it alone, with the same results.  Every block must start 16-byte aligned (H * N_i * d is a
  * multiple of 8 elements, which d = 128 guarantees).  All sizes are checked before the first
- * launch.  The workspace is sized for the largest sequence; the sequences run one after
- * another on `stream`. */
+ * launch.  The sequences are taken longest first in groups: a group takes the next sequence
+ * while its heads padded to its longest stay within twice their own padded size, or below
+ * 2^20 padded token-heads; each group is one prologue and one attention launch (the kernels
+ * read every head's own length from a table), so a batch of short sequences is a single
+ * launch of each kernel.  The workspace is sized for the largest group, plus the table,
+ * which is uploaded through a library-owned page-locked host buffer. */
 sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int nseq, const int *seqlens,
                              int H, int d, float sm_scale, int causal, void *stream);
 

@@ -36,3 +36,32 @@ def test_varlen_equals_per_sequence_calls(oracle, libsa, cuda_ok, causal):
                            causal=causal)
     assert np.abs(got - ref).max() <= O_MAX_ABS
     assert cosine(got, ref) >= O_MIN_COS
+
+
+def _check_against_own_calls(libsa, lens, H, causal, seed):
+    seqs = [make_inputs(1, H, n, seed=seed + i, outliers=(i % 2 == 0))[:3] for i, n in enumerate(lens)]
+    packed = [torch.cat([to_dev_bf16(s[t]).reshape(-1) for s in seqs]) for t in range(3)]
+    o = libsa.sa_attn_fwd_varlen(*packed, lens, H, causal=causal)
+    assert libsa.sa_get_device_status() == 0
+    off = 0
+    for n, (q, k, v) in zip(lens, seqs):
+        qd, kd, vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+        ref = libsa.sa_attn_fwd_causal(qd, kd, vd) if causal else libsa.sa_attn_fwd(qd, kd, vd)
+        got = o[off:off + H * n * 128].reshape(1, H, n, 128)
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), n
+        off += H * n * 128
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_64_short_sequences_one_launch_each_equal_own_call(libsa, cuda_ok, causal):
+    """64 sequences of 1 to 512 tokens: one group, i.e. one prologue and one attention
+    launch for the whole batch; every sequence bit for bit as its own call."""
+    lens = [int(n) for n in np.random.default_rng(77).integers(1, 513, size=64)]
+    lens[0], lens[1] = 1, 512
+    _check_against_own_calls(libsa, lens, 2, causal, seed=3000)
+
+
+def test_varlen_groups_of_mixed_lengths(libsa, cuda_ok):
+    """One long sequence and forty short ones: the padding rule splits them into two groups
+    (the long one with the first 25 short ones, then the rest); results unchanged."""
+    _check_against_own_calls(libsa, [40000] + [1000] * 40, 1, False, seed=3100)
