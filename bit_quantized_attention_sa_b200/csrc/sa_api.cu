@@ -271,7 +271,9 @@ static sa_status attn_fwd_device(const void *q, const void *k, const void *v, vo
 //
 // sa_attn_fwd_host: the heads (b, h) are independent, so the B*H heads are cut into chunks
 // of consecutive heads; the upload of chunk c+1 and the download of chunk c-1 run on two
-// library streams while chunk c is computed on the caller's stream.  Two staging slots per
+// library streams while chunk c is computed on the caller's stream.  Chunk c holds at most
+// c + 1 heads (then the full chunk size): the first upload, which nothing overlaps, stays
+// one head long, and each later upload still fits under the computation before it.  Two staging slots per
 // device alternate between chunks; events order each slot's reuse:
 //   upload(c)   waits compute(c-2)   (its inputs were read)
 //   compute(c)  waits upload(c) and download(c-2) (its output slot was copied out)
@@ -344,9 +346,9 @@ static sa_status attn_fwd_host_pipeline(const void *q, const void *k, const void
     if (cudaEventRecord(P.entry, st) != cudaSuccess || cudaStreamWaitEvent(P.h2d, P.entry, 0) != cudaSuccess)
         return SA_ERR_CUDA;
     int last[2] = {0, 0};
-    for (int64_t h0 = 0, c = 0; h0 < BH; h0 += hc, ++c) {
+    for (int64_t h0 = 0, c = 0, hn = 0; h0 < BH; h0 += hn, ++c) {
         const int i = int(c & 1);
-        const int64_t hn = std::min<int64_t>(hc, BH - h0);
+        hn = std::min<int64_t>(std::min<int64_t>(hc, c + 1), BH - h0);
         const size_t nb = size_t(hn) * head_bytes, off = size_t(h0) * head_bytes;
         uint8_t *base = static_cast<uint8_t *>(P.buf) + size_t(i) * slot;
         uint8_t *dq = base, *dk = base + t_bytes, *dv = base + 2 * t_bytes, *dout = base + 3 * t_bytes;

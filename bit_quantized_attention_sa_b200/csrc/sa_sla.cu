@@ -14,10 +14,11 @@
 // d features of a row, or elu + 1.
 //
 // Kernels, over groups of heads whose states fit a bounded workspace:
-//   sla_state_kernel      one CTA per (head, 64-key block), fp32 on the CUDA cores: H_j
-//                         (128 x 128) and Z_j, stored as one 128 x 136 block whose column
-//                         128 is Z_j (columns 129-135 zero), so that the apply step gets the
-//                         normaliser from the same product as the numerator.
+//   sla_state_mma_kernel  one CTA per (head, 64-key block): H_j (128 x 128) and Z_j as one
+//                         TF32 tcgen05 GEMM of phi(K_j)^T with [V_j | 1], phi split into hi +
+//                         lo; stored as one 128 x 136 block whose column 128 is Z_j (columns
+//                         129-135 zero), so that the apply step gets the normaliser from the
+//                         same product as the numerator.
 //   sla_marginal_kernel   the 0/1 matrix C[i][j] = (class == 1) in fp32.
 //   sla_sum_mma_kernel    A_i = sum_j C[i][j] H_j for every query block: a TF32 tcgen05 GEMM
 //                         (K = key blocks) with the states split into hi + lo terms.
@@ -41,98 +42,203 @@ namespace {
 constexpr int kStateCols = 136;                      // H_j columns, then Z_j, then zeros
 constexpr int kStateFloats = kD * kStateCols;        // 17408 per key (or query) block
 
-// phi of one 128-feature row held by a warp, 4 features per lane (features 4 lane .. +3).
-__device__ __forceinline__ void phi_row_warp(float (&x)[4], int phi)
+__device__ int g_sla_status;  // 0 = OK, 6 = a bounded wait expired
+
+// A wait bounded by time alone (not by the abort flag): used to let this CTA's own
+// copies and MMAs land before it frees its memory.
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity)
 {
-    if (phi == 0) {
-        float m = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > SA_WAIT_LIMIT_NS) return false;
+    return true;
+}
+
+// hi keeps the sign, exponent and top 10 mantissa bits (exact in TF32); lo = x - hi exactly.
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+// ---- the per-block states on the tensor cores
+// H_j[a][b] = sum_{t in block j} phi(k_t)[a] [v_t, 1, 0...][b]: M = 128 features a, N = 144
+// (the 128 value channels, the ones column that gives Z_j, zeros), K = the block's 64
+// tokens; kind::tf32 with phi split into hi + lo (two products; v is bf16, exact in TF32),
+// fp32 accumulation in tensor memory.  Both operands are MN-major (feature a, resp. channel
+// b, contiguous) in the 128-byte swizzle of 32-byte granules: an atom is 4 token rows of 128
+// bytes (32 values), granule g of row t at granule position g ^ (t & 3); atom columns of
+// 64 rows are 8 KB apart, 4-row groups 512 bytes apart.
+//   all 8 warps  token t = 8 * warp + lane / 4 and atom column c = lane % 4 (32 features
+//                or channels): phi over the row's 128 features (the 4 lanes of a token
+//                exchange the maximum and the sum), phi hi/lo and v into the tiles; column
+//                4 of v holds the ones column.
+//   thread 0     the 16 MMAs, committed to one barrier.
+//   all 8 warps  the epilogue: warp w reads tensor-memory lanes 32 (w % 4) .., columns
+//                0-63 (w < 4) or 64-135 (w >= 4), and stores the state rows.
+namespace stm {
+constexpr uint32_t kCol = 64 * 128;                                 // one atom column, 8 KB
+constexpr uint32_t kOffPhiHi = 0, kOffPhiLo = 4 * kCol, kOffV = 8 * kCol;  // V: 5 columns
+constexpr uint32_t kOffBar = kOffV + 5 * kCol;
+constexpr uint32_t kSmem = kOffBar + 16 + 1024;
+constexpr int kN = 144;
+static_assert(kSmem <= 116 * 1024, "two CTAs per SM");
+}  // namespace stm
+
+// byte offset of the 8-value granule g of token row t in an MN-major atom column
+__device__ __forceinline__ uint32_t mn32_off(int t, int g)
+{
+    return uint32_t(t >> 2) * 512u + uint32_t(t & 3) * 128u + (uint32_t(g ^ (t & 3)) << 5);
+}
+
+// grid (nk, heads), 256 threads, stm::kSmem bytes (two CTAs per SM).
+__global__ void __launch_bounds__(256, 2)
+    sla_state_mma_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, int N, int nk, int phi,
+                         float *__restrict__ state)
+{
+    using namespace stm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int j = blockIdx.x, bh = blockIdx.y;
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + kOffBar + 8);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffBar + 12);
+    const uint32_t bar = sbase + kOffBar;
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(sbase + kOffBar + 8, 256);
+
+    // ---- operands: token t, atom column c (features / channels 32c .. 32c + 31)
+    {
+        const int t = 8 * warp + (lane >> 2), c = lane & 3;
+        const int64_t tok = int64_t(j) * kKBlk + t;
+        const bool valid = tok < N;
+        const int64_t row = (int64_t(bh) * N + (valid ? tok : 0)) * kD + 32 * c;
+        float x[32];
+        uint4 vr[4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        float s = 0.0f;
+        for (int u = 0; u < 4; ++u) {
+            const uint4 kw = valid ? __ldg(reinterpret_cast<const uint4 *>(k + row) + u) : make_uint4(0u, 0u, 0u, 0u);
+            vr[u] = valid ? __ldg(reinterpret_cast<const uint4 *>(v + row) + u) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t w4[4] = {kw.x, kw.y, kw.z, kw.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            x[e] = expf(x[e] - m);
-            s += x[e];
+            for (int e = 0; e < 4; ++e) {
+                x[8 * u + 2 * e] = __uint_as_float(w4[e] << 16);
+                x[8 * u + 2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+            }
+        }
+        if (phi == 0) {
+            float m = x[0];
+#pragma unroll
+            for (int f = 1; f < 32; ++f) m = fmaxf(m, x[f]);
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            float sum = 0.0f;
+#pragma unroll
+            for (int f = 0; f < 32; ++f) {
+                x[f] = expf(x[f] - m);
+                sum += x[f];
+            }
+            sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+            sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+#pragma unroll
+            for (int f = 0; f < 32; ++f) x[f] = __fdiv_rn(x[f], sum);
+        } else {
+#pragma unroll
+            for (int f = 0; f < 32; ++f) x[f] = x[f] > 0.0f ? x[f] + 1.0f : expf(x[f]);
+        }
+        if (!valid) {
+#pragma unroll
+            for (int f = 0; f < 32; ++f) x[f] = 0.0f;  // rows past N take no part
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        for (int g = 0; g < 4; ++g) {
+            float4 h0, h1, l0, l1, v0, v1;
+            h0 = make_float4(tf32_hi(x[8 * g]), tf32_hi(x[8 * g + 1]), tf32_hi(x[8 * g + 2]), tf32_hi(x[8 * g + 3]));
+            h1 = make_float4(tf32_hi(x[8 * g + 4]), tf32_hi(x[8 * g + 5]), tf32_hi(x[8 * g + 6]), tf32_hi(x[8 * g + 7]));
+            l0 = make_float4(x[8 * g] - h0.x, x[8 * g + 1] - h0.y, x[8 * g + 2] - h0.z, x[8 * g + 3] - h0.w);
+            l1 = make_float4(x[8 * g + 4] - h1.x, x[8 * g + 5] - h1.y, x[8 * g + 6] - h1.z, x[8 * g + 7] - h1.w);
+            const uint32_t w4[4] = {vr[g].x, vr[g].y, vr[g].z, vr[g].w};
+            v0 = make_float4(__uint_as_float(w4[0] << 16), __uint_as_float(w4[0] & 0xFFFF0000u),
+                             __uint_as_float(w4[1] << 16), __uint_as_float(w4[1] & 0xFFFF0000u));
+            v1 = make_float4(__uint_as_float(w4[2] << 16), __uint_as_float(w4[2] & 0xFFFF0000u),
+                             __uint_as_float(w4[3] << 16), __uint_as_float(w4[3] & 0xFFFF0000u));
+            const uint32_t off = uint32_t(c) * kCol + mn32_off(t, g);
+            *reinterpret_cast<float4 *>(smem + kOffPhiHi + off) = h0;
+            *reinterpret_cast<float4 *>(smem + kOffPhiHi + off + 16) = h1;
+            *reinterpret_cast<float4 *>(smem + kOffPhiLo + off) = l0;
+            *reinterpret_cast<float4 *>(smem + kOffPhiLo + off + 16) = l1;
+            *reinterpret_cast<float4 *>(smem + kOffV + off) = v0;
+            *reinterpret_cast<float4 *>(smem + kOffV + off + 16) = v1;
+        }
+        // V column 4 (channels 128-159): the ones column 128 (zero past N), then zeros
+        const float one = valid ? 1.0f : 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = __fdiv_rn(x[e], s);
-    } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = x[e] > 0.0f ? x[e] + 1.0f : expf(x[e]);
+        for (int g = 0; g < 4; ++g) {
+            if (g != c) continue;  // the token's 4 lanes write one granule each
+            const uint32_t off = 4u * kCol + mn32_off(t, g);
+            *reinterpret_cast<float4 *>(smem + kOffV + off) = make_float4(g == 0 ? one : 0.0f, 0.0f, 0.0f, 0.0f);
+            *reinterpret_cast<float4 *>(smem + kOffV + off + 16) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
     }
-}
-
-// Loads row t of a head (bf16, 128 features) into 4 floats per lane; zeros past N.
-__device__ __forceinline__ void load_row4(const uint16_t *base, int64_t t, int64_t N, int lane, float (&x)[4])
-{
-    if (t < N) {
-        const uint2 w = *reinterpret_cast<const uint2 *>(base + t * kD + 4 * lane);
-        x[0] = __uint_as_float(w.x << 16);
-        x[1] = __uint_as_float(w.x & 0xFFFF0000u);
-        x[2] = __uint_as_float(w.y << 16);
-        x[3] = __uint_as_float(w.y & 0xFFFF0000u);
-    } else {
-        x[0] = x[1] = x[2] = x[3] = 0.0f;
-    }
-}
-
-// grid (nk, BH), 256 threads, dynamic shared memory 2 x 64 x 128 floats.
-__global__ void __launch_bounds__(256)
-    sla_state_kernel(const uint16_t *__restrict__ k, const uint16_t *__restrict__ v, int N, int nk, int phi,
-                     float *__restrict__ state)
-{
-    extern __shared__ __align__(16) float sm[];
-    float *pk = sm;               // [64][128] phi(k) rows of the block (zero past N)
-    float *vv = sm + kKBlk * kD;  // [64][128] v rows
-    const int64_t bh = blockIdx.y;
-    const int j = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint16_t *kh = k + bh * int64_t(N) * kD, *vh = v + bh * int64_t(N) * kD;
-    for (int t = warp; t < kKBlk; t += 8) {
-        const int64_t tok = int64_t(j) * kKBlk + t;
-        float x[4], y[4];
-        load_row4(kh, tok, N, lane, x);
-        load_row4(vh, tok, N, lane, y);
-        if (tok < N) phi_row_warp(x, phi);
-        *reinterpret_cast<float4 *>(pk + t * kD + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
-        *reinterpret_cast<float4 *>(vv + t * kD + 4 * lane) = make_float4(y[0], y[1], y[2], y[3]);
-    }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // H[a][c] for a in [8 ty, 8 ty + 8), c in [8 tx, 8 tx + 8), over the block's 64 tokens
-    const int ty = tid >> 4, tx = tid & 15;
-    float acc[8][8];
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) {
+        const uint32_t idesc = idesc_tf32_f32(128, kN, true, true);
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = 0.0f;
-    for (int t = 0; t < kKBlk; ++t) {
-        const float4 p0 = *reinterpret_cast<const float4 *>(pk + t * kD + 8 * ty);
-        const float4 p1 = *reinterpret_cast<const float4 *>(pk + t * kD + 8 * ty + 4);
-        const float4 v0 = *reinterpret_cast<const float4 *>(vv + t * kD + 8 * tx);
-        const float4 v1 = *reinterpret_cast<const float4 *>(vv + t * kD + 8 * tx + 4);
-        const float pa[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        const float vc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-        for (int a = 0; a < 8; ++a)
-#pragma unroll
-            for (int c = 0; c < 8; ++c) acc[a][c] = fmaf(pa[a], vc[c], acc[a][c]);
+        for (int kk = 0; kk < kKBlk / 8; ++kk) {
+            const uint64_t bd = sdesc_mn32(sbase + kOffV + 1024u * kk, kCol, 512);
+            mma_tf32(tmem, sdesc_mn32(sbase + kOffPhiHi + 1024u * kk, kCol, 512), bd, idesc, kk > 0);
+            mma_tf32(tmem, sdesc_mn32(sbase + kOffPhiLo + 1024u * kk, kCol, 512), bd, idesc, 1);
+        }
+        tc_commit(bar);
     }
-    float *out = state + (bh * nk + j) * int64_t(kStateFloats);
+    bool ok = mbar_wait(bar, 0, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+        tc_fence_after();
+        const int a = 32 * (warp & 3) + lane;
+        const uint32_t ta = tmem + (uint32_t(32 * (warp & 3)) << 16);
+        float *out = state + ((int64_t(bh) * nk + j) * kD + a) * kStateCols;
+        uint32_t r[32];
+        if (warp < 4) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+                tmem_ld32_wait(ta + c0, r);
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-        float *row = out + (8 * ty + a) * kStateCols + 8 * tx;
-        *reinterpret_cast<float4 *>(row) = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-        *reinterpret_cast<float4 *>(row + 4) = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(out + c0 + e) =
+                        make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                                    __uint_as_float(r[e + 3]));
+            }
+        } else {
+            for (int c0 = 64; c0 < 128; c0 += 32) {
+                tmem_ld32_wait(ta + c0, r);
+#pragma unroll
+                for (int e = 0; e < 32; e += 4)
+                    *reinterpret_cast<float4 *>(out + c0 + e) =
+                        make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                                    __uint_as_float(r[e + 3]));
+            }
+            uint32_t r8[8];
+            tmem_ld8_wait(ta + 128, r8);  // Z_j, then the zero columns 129-135
+            *reinterpret_cast<float4 *>(out + 128) =
+                make_float4(__uint_as_float(r8[0]), __uint_as_float(r8[1]), __uint_as_float(r8[2]), __uint_as_float(r8[3]));
+            *reinterpret_cast<float4 *>(out + 132) =
+                make_float4(__uint_as_float(r8[4]), __uint_as_float(r8[5]), __uint_as_float(r8[6]), __uint_as_float(r8[7]));
+        }
+    } else if (lane == 0) {
+        *abort_flag = 1;
+        atomicExch(&g_sla_status, 6);
     }
-    if (tid < kD) {
-        // column 128: Z_j[a] = sum over the block's tokens of phi(k_t)[a]; columns 129-135 zero
-        float z = 0.0f;
-        for (int t = 0; t < kKBlk; ++t) z += pk[t * kD + tid];
-        float *row = out + tid * kStateCols + kD;
-        *reinterpret_cast<float4 *>(row) = make_float4(z, 0.0f, 0.0f, 0.0f);
-        *reinterpret_cast<float4 *>(row + 4) = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
+    if (threadIdx.x == 0 && !drain_wait(bar, 0)) atomicExch(&g_sla_status, 6);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // ---- the class-weighted state sum on the tensor cores
@@ -173,18 +279,6 @@ constexpr uint32_t kSmem = kOffMisc + 16 + 1024;  // + slack for the 1024-byte a
 static_assert(kOffB % 1024 == 0 && kABytes % 1024 == 0 && kBBytes % 1024 == 0, "swizzle atoms");
 static_assert(kSmem <= 232448, "shared memory");
 }  // namespace summ
-
-__device__ int g_sla_status;  // 0 = OK, 6 = a bounded wait expired
-
-// A wait bounded by time alone (not by the abort flag): used to let this CTA's own
-// copies and MMAs land before it frees its memory.
-__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity)
-{
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > SA_WAIT_LIMIT_NS) return false;
-    return true;
-}
 
 // grid (ceil(nq / nt), 17408 / 128, BH), summ::kThreads threads, summ::kSmem bytes.
 // nt: query blocks per tile, a multiple of 16 in [16, 256].
@@ -377,9 +471,6 @@ constexpr uint32_t kSmem = kOffMisc + 16 + 1024;
 constexpr uint32_t kColAcc1 = 0, kColAcc2 = 256;  // D1: 144 columns; D2: 128 columns
 static_assert(kOffAHi % 1024 == 0 && kSmem <= 232448, "apply shared memory");
 }  // namespace appm
-
-// hi keeps the sign, exponent and top 10 mantissa bits (exact in TF32); lo = x - hi exactly.
-__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
 
 // Writes 4 consecutive K values (chunk c of 8 in a 128-byte row) of row r of a K-major,
 // 128-byte swizzled atom, as hi and lo.
@@ -664,10 +755,9 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const size_t state_smem = size_t(2) * kKBlk * kD * sizeof(float);
     if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        if ((e = cudaFuncSetAttribute(sla_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      int(state_smem))) != cudaSuccess ||
+        if ((e = cudaFuncSetAttribute(sla_state_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      int(stm::kSmem))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_sum_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       int(summ::kSmem))) != cudaSuccess ||
             (e = cudaFuncSetAttribute(sla_apply_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -687,7 +777,7 @@ cudaError_t launch_sla_linear(const void *q, const void *k, const void *v, const
     const int nt = ((nq + ntiles - 1) / ntiles + 15) / 16 * 16;
     for (int64_t h0 = 0; h0 < s.BH(); h0 += G) {
         const int64_t g = s.BH() - h0 < G ? s.BH() - h0 : G;
-        sla_state_kernel<<<dim3(unsigned(nk), unsigned(g)), 256, state_smem, st>>>(
+        sla_state_mma_kernel<<<dim3(unsigned(nk), unsigned(g)), 256, stm::kSmem, st>>>(
             static_cast<const uint16_t *>(k) + h0 * tok, static_cast<const uint16_t *>(v) + h0 * tok, N, nk, phi,
             state);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

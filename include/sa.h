@@ -154,9 +154,11 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
 
 /* Full forward on HOST buffers: q, k, v, o bf16 [B,H,N,d] and block_mask (or NULL) in host
  * memory, page-locked for the copies to overlap (pageable memory works but serialises).
- * The B*H heads are independent, so they are processed in chunks of consecutive heads:
- * the upload of chunk c+1 and the download of chunk c-1 run on two library-owned streams
- * while chunk c runs sa_attn_fwd's prologue and kernel on `stream`.  The call returns
+ * The B*H heads are independent, so they are processed in chunks of consecutive heads
+ * (one head first, then growing by one head per chunk up to about 64 MB of q, so that the
+ * first upload, which nothing overlaps, is short): the upload of chunk c+1 and the
+ * download of chunk c-1 run on two library-owned streams while chunk c runs sa_attn_fwd's
+ * prologue and kernel on `stream`.  The call returns
  * after enqueueing; the work is complete when `stream` reaches the point after the call
  * (o is then filled), and q, k, v, o and block_mask must stay valid until then.  Device staging (two chunks) is library-owned, per device and
  * grow-only, like the workspace.  Calls for the same device from several host threads
