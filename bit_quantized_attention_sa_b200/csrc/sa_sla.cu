@@ -636,7 +636,12 @@ __global__ void __launch_bounds__(appm::kThreads, 1)
                 m = fmaxf(m, fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w)));
             }
         }
-        auto phi1 = [&](float v) -> float { return phi == 0 ? expf(v - m) : (v > 0.0f ? v + 1.0f : expf(v)); };
+        // exponentials as ex2.approx of the argument times log2(e) (a few ulp, far inside
+        // the branch's 1e-4 bound)
+        constexpr float kL2e = 1.4426950408889634f;
+        auto phi1 = [&](float v) -> float {
+            return phi == 0 ? ex2_approx((v - m) * kL2e) : (v > 0.0f ? v + 1.0f : ex2_approx(v * kL2e));
+        };
 #pragma unroll
         for (int c4 = 0; c4 < kD / 4; ++c4) {
             float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
