@@ -84,6 +84,8 @@ static sa_status check_shape(int B, int H, int N, int d, Shape *s)
     s->N = N;
     // TMA row coordinates and tile indices are 32-bit
     if (s->BH() > INT_MAX / 8 || s->BH() * s->Npad() > INT_MAX) return SA_ERR_INVALID_ARG;
+    // the heads are a grid dimension (y) of the prologue kernels
+    if (s->BH() > 65535) return SA_ERR_UNSUPPORTED;
     return SA_OK;
 }
 
@@ -753,6 +755,7 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
         while (g0 + cnt < nseq) {
             const int64_t own2 = own + padded_len(seqlens[ord[g0 + cnt]]), pad2 = int64_t(cnt + 1) * pmax;
             if (pad2 > 2 * own2 && pad2 * H > (int64_t(1) << 20)) break;
+            if (int64_t(cnt + 1) * H > 65535) break;  // a group's heads are a grid dimension
             own = own2;
             ++cnt;
         }

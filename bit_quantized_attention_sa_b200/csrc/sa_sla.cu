@@ -742,7 +742,8 @@ static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 static int64_t chunk_heads(const Shape &s)
 {
     const int64_t per = int64_t(head_state_bytes(s) + head_sum_bytes(s) + head_c_bytes(s));
-    const int64_t g = int64_t(kChunkBudget) / per;
+    int64_t g = int64_t(kChunkBudget) / per;
+    if (g > 65535) g = 65535;  // the group is a grid dimension of every launch
     return g < 1 ? 1 : (g > s.BH() ? s.BH() : g);
 }
 

@@ -31,7 +31,8 @@
  *     that sa_attn_fwd and sa_attn_fwd_causal also take d = 64: they zero-pad q, k, v to 128
  *     channels in the workspace and copy out o's first 64, which gives exactly the d = 64
  *     definition (zero channels add nothing to S and leave every scale and code unchanged).
- *     Npad = 128 * ceil(N/128); nq = ceil(N/128); nk = ceil(N/64).
+ *     Npad = 128 * ceil(N/128); nq = ceil(N/128); nk = ceil(N/64).  B * H <= 65535 (the
+     heads are a grid dimension of the prologue kernels), else SA_ERR_UNSUPPORTED.
  *   - Device pointers are owned by the caller; the library never frees them.  All
  *     pointers must be 16-byte aligned.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
@@ -70,7 +71,7 @@ extern "C" {
 typedef enum {
     SA_OK = 0,
     SA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, size overflow */
-    SA_ERR_UNSUPPORTED = 2,    /* d != 128, or no sm_100 device */
+    SA_ERR_UNSUPPORTED = 2,    /* d != 128, B * H > 65535, or no sm_100 device */
     SA_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
     SA_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed */
     SA_ERR_OOM = 5,            /* the library workspace could not be allocated */

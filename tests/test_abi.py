@@ -46,6 +46,7 @@ ODD = ctypes.c_void_p((1 << 20) + 8)  # misaligned
     ((FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 128, 0.088, None, None), 1),     # N = 0
     ((FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, 0.088, None, None), 1),   # B = 0
     ((FAKE, FAKE, FAKE, FAKE, 1 << 20, 1 << 10, 128, 128, 0.088, None, None), 1),  # overflow
+    ((FAKE, FAKE, FAKE, FAKE, 2, 32768, 128, 128, 0.088, None, None), 2),  # B*H > 65535
     ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0.0, None, None), 1),     # sm_scale <= 0
     ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, float("nan"), None, None), 1),
 ])
