@@ -520,7 +520,7 @@ def main():
     ops_rank = w.dense_ops
     value = whole_job_tops(ops_rank, world, t_step)
     achieved = ops_rank / t_attn / 1e12
-    kernel = "attn_fwd_kernel" if w.mask_density is not None else "attn_pairs_kernel"
+    kernel = "attn_mpairs_kernel" if w.mask_density is not None else "attn_pairs_kernel"
     traffic = recorded_traffic(kernel, w.name)
 
     cpu = None

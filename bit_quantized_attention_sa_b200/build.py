@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsa.so")
 SOURCES = ["sa_api.cu", "sa_prologue.cu", "sa_attn.cu", "sa_mask.cu", "sa_w8a8.cu", "sa_sla.cu", "sa_peak.cu"]
-HEADERS = ["sa_ptx.cuh", "sa_internal.h", "sa_attn_pairs.cuh"]
+HEADERS = ["sa_ptx.cuh", "sa_internal.h", "sa_attn_pairs.cuh", "sa_attn_mpairs.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -2,7 +2,7 @@
 // Included by sa_attn.cu inside its anonymous namespace (shares its constants, the device
 // status word and the helpers above the include).
 //
-// Same computation as attn_fwd_kernel without a keep mask (every 64-key block kept, steps
+// The attention forward without a keep mask (every 64-key block kept, steps
 // of two consecutive blocks; "AIGC weekend special 5.10" section 1.2 Method item (1),
 // FlashAttention's tiled online softmax), organised for latency hiding:
 //   * A CTA takes a pair of 128-query tiles (A, B) of one head.  Both read the same K/V
@@ -21,7 +21,8 @@
 //     softmax warpgroups raise theirs to 232 (a whole 128-key row of S in registers) and
 //     the third lowers its to 40 (setmaxnreg): 2*232 + 40 <= 3*168.
 // Tensor memory: S [0,128), O_A [128,272), O_B [272,416).
-// Every mbarrier wait is bounded, as in attn_fwd_kernel.
+// Every mbarrier wait is bounded (sa_ptx.cuh); on expiry the kernel records the device
+// timeout status and exits.
 
 namespace pairs {
 
