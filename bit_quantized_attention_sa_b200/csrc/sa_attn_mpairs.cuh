@@ -19,7 +19,8 @@
 //     from them; the producer takes the blocks from the bitmasks and records each stage's
 //     block indices, which the softmax reads for the K scales and the valid keys.
 //   * A tile with no kept block writes zero rows (or the addend) and takes no part in the
-//     barrier sequence; a pair with none at all is skipped by every role.
+//     barrier sequence; a pair with none at all is skipped by every role but the softmax
+//     warpgroups, which write its rows.
 // Every mbarrier wait is bounded, as in the other attention kernels.
 
 namespace mpairs {
@@ -382,7 +383,7 @@ __global__ void __launch_bounds__(pairs::kThreads, 1)
             nB = __shfl_sync(0xffffffffu, nB, 0);
             __syncwarp();
             if (lane == 0) mbar_arrive(ebar(2 + int(pi & 1)));
-            if (nA + nB == 0) continue;
+            // a pair with no kept block at all still writes its rows (below, n == 0)
             const int qt = qa + t, n = t ? nB : nA, mn = min(nA, nB), total = nA + nB;
             const int qrow = qt * 128 + row;
             if (n == 0) {

@@ -104,6 +104,33 @@ def test_all_ones_mask_is_bit_identical_to_no_mask(libsa, cuda_ok):
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
 
 
+def test_masks_with_empty_tile_pairs(oracle, libsa, cuda_ok):
+    """Query tiles are processed two at a time: an all-zero mask gives exact zeros, and a
+    mask that empties whole pairs of tiles (and one tile of another pair) gives zeros there
+    and the oracle's rows elsewhere."""
+    N = 1000  # 8 query tiles, the last ragged
+    q, k, v, _ = make_inputs(1, 2, N, seed=13, outliers=True)
+    qd, kd, vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+    nq, nk = 8, 16
+    zeros = torch.zeros((1, 2, nq, nk), dtype=torch.uint8, device="cuda")
+    o = libsa.sa_attn_fwd(qd, kd, vd, block_mask=zeros)
+    assert libsa.sa_get_device_status() == 0
+    assert not o.float().abs().max().item()
+    m = (np.random.default_rng(5).random((1, 2, nq, nk)) < 0.3).astype(np.uint8)
+    m[0, 0, 2:4] = 0   # the pair (2, 3) of head 0
+    m[0, 1, 4:6] = 0   # the pair (4, 5) of head 1
+    m[0, 1, 7] = 0     # tile 7 of head 1 (its pair partner 6 keeps blocks)
+    m[0, 1, 6, 3] = 1
+    o = libsa.sa_attn_fwd(qd, kd, vd, block_mask=torch.from_numpy(m).cuda())
+    assert libsa.sa_get_device_status() == 0
+    rows = all_rows(1, 2, N)
+    got = gpu_rows(o, rows)
+    ref = oracle.attn_rows(oracle.quantize_qk(q, k), oracle.quantize_v(v), N, sm_scale(), rows, m, 2)
+    compare(got, ref, "empty pairs")
+    for bh, lo, hi in ((0, 256, 512), (1, 512, 768), (1, 896, N)):
+        assert not o[0, bh, lo:hi].float().abs().max().item()
+
+
 def test_diagonal_mask_matches_exact_on_kept_keys(oracle, libsa, cuda_ok):
     N = 1024
     q, k, v, _ = make_inputs(1, 1, N, seed=11)
