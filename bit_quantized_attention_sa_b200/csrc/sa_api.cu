@@ -479,11 +479,19 @@ static sa_status attn_fwd_d64(const void *q, const void *k, const void *v, void 
     return launch_unpad_heads(po, rows, o, st) == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
 
-static sa_status check_d64_call(int B, int H, int N, float sm_scale, std::initializer_list<const void *> ptrs)
+// A keep mask row of a masked attention call holds at most kMaskedAttnMaxKeyBlocks blocks.
+static sa_status check_mask_len(const Shape &s, const void *mask)
+{
+    return mask && s.nk() > kMaskedAttnMaxKeyBlocks ? SA_ERR_UNSUPPORTED : SA_OK;
+}
+
+static sa_status check_d64_call(int B, int H, int N, float sm_scale, std::initializer_list<const void *> ptrs,
+                                const void *mask)
 {
     Shape s;
     sa_status r = check_shape(B, H, N, kD, &s);
     if (r != SA_OK) return r;
+    if ((r = check_mask_len(s, mask)) != SA_OK) return r;
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs(ptrs)) != SA_OK) return r;
     return check_device();
@@ -493,7 +501,7 @@ sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int 
                       int N, int d, float sm_scale, const uint8_t *block_mask, void *stream)
 {
     if (d == kD / 2) {
-        const sa_status r = check_d64_call(B, H, N, sm_scale, {q, k, v, o});
+        const sa_status r = check_d64_call(B, H, N, sm_scale, {q, k, v, o}, block_mask);
         return r != SA_OK ? r
                           : attn_fwd_d64(q, k, v, o, B, H, N, sm_scale, block_mask, false,
                                          static_cast<cudaStream_t>(stream));
@@ -503,6 +511,7 @@ sa_status sa_attn_fwd(const void *q, const void *k, const void *v, void *o, int 
     if (r != SA_OK) return r;
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
+    if ((r = check_mask_len(s, block_mask)) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     return attn_fwd_device(q, k, v, o, s, sm_scale, block_mask, static_cast<cudaStream_t>(stream));
 }
@@ -515,6 +524,7 @@ sa_status sa_attn_fwd_host(const void *q, const void *k, const void *v, void *o,
     if (r != SA_OK) return r;
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
+    if ((r = check_mask_len(s, block_mask)) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     return attn_fwd_host_pipeline(q, k, v, o, s, sm_scale, block_mask, static_cast<cudaStream_t>(stream));
 }
@@ -530,6 +540,7 @@ sa_status sa_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale, const 
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs({q_i8, k_i8, v_fp8_t, o})) != SA_OK) return r;
     if (!q_scale || !k_scale || !v_scale) return SA_ERR_INVALID_ARG;
+    if ((r = check_mask_len(s, block_mask)) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     return attention_core(q_i8, q_scale, k_i8, k_scale, v_fp8_t, v_scale, o, s, sm_scale,
                           block_mask, static_cast<cudaStream_t>(stream));
@@ -696,7 +707,7 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
                              float sm_scale, const uint8_t *block_mask, void *stream)
 {
     if (d == kD / 2) {
-        const sa_status r = check_d64_call(B, H, N, sm_scale, {q, k, v, o});
+        const sa_status r = check_d64_call(B, H, N, sm_scale, {q, k, v, o}, block_mask);
         return r != SA_OK ? r
                           : attn_fwd_d64(q, k, v, o, B, H, N, sm_scale, block_mask, true,
                                          static_cast<cudaStream_t>(stream));
@@ -706,6 +717,7 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
     if (r != SA_OK) return r;
     if (!(sm_scale > 0.0f) || !std::isfinite(sm_scale)) return SA_ERR_INVALID_ARG;
     if ((r = check_ptrs({q, k, v, o})) != SA_OK) return r;
+    if ((r = check_mask_len(s, block_mask)) != SA_OK) return r;
     if ((r = check_device()) != SA_OK) return r;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // without a keep mask the pair kernel runs the causal pattern itself

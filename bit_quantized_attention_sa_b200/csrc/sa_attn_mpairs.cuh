@@ -25,7 +25,7 @@
 
 namespace mpairs {
 
-constexpr int kMaxBlocks = 16384;                     // key blocks per mask row (N <= 1,048,576)
+constexpr int kMaxBlocks = kMaskedAttnMaxKeyBlocks;  // key blocks per mask row (N <= 1,048,576)
 constexpr int kWords = kMaxBlocks / 32;               // bitmask words per tile
 constexpr uint32_t kOffInfo = pairs::kOffMisc + 16;  // int2 [kStages]: the blocks of each stage
 constexpr uint32_t kOffEntBar = kOffInfo + 8 * pairs::kStages;  // entry full [2], empty [2]

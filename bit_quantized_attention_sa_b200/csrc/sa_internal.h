@@ -78,6 +78,7 @@ cudaError_t launch_debug_qk_s32(const CUtensorMap &tm_q, const CUtensorMap &tm_k
 cudaError_t launch_debug_wait_timeout(int timeout_us, cudaStream_t st);
 // ---- block-mask producer (sa_mask.cu)
 constexpr int kMaskMaxKeyBlocks = 4096;  // key blocks per mask row the selector sorts in shared memory
+constexpr int kMaskedAttnMaxKeyBlocks = 16384;  // key blocks per mask row of a masked attention call
 cudaError_t launch_pool_qk(const void *q, const void *k, const Shape &s, float *qbar, float *kbar,
                            cudaStream_t st);
 // Causal block mask: out[bh][i][j] = (j <= 2i + 1) && (user == null || user[bh][i][j] != 0).

@@ -42,7 +42,8 @@
  *     untouched.  Launch failures return SA_ERR_CUDA.  Device-side bounded waits that
  *     expire set a device status word read by sa_get_device_status.
  *   - Block mask: uint8 [B,H,nq,nk], nonzero keeps the (128-query x 64-key) block; NULL
- *     keeps every block.  Masked blocks are neither loaded nor computed.
+ *     keeps every block.  Masked blocks are neither loaded nor computed.  With a mask,
+ *     nk <= 16384 (N <= 1,048,576), else SA_ERR_UNSUPPORTED.
  *   - Library workspace.  The entry points marked "uses the library workspace" keep their
  *     intermediates (quantised Q/K/V, scales, partial sums, masks, SLA states) in ONE
  *     buffer per device, owned by the library and grown on demand.  Growing it

@@ -47,6 +47,8 @@ ODD = ctypes.c_void_p((1 << 20) + 8)  # misaligned
     ((FAKE, FAKE, FAKE, FAKE, 0, 1, 128, 128, 0.088, None, None), 1),   # B = 0
     ((FAKE, FAKE, FAKE, FAKE, 1 << 20, 1 << 10, 128, 128, 0.088, None, None), 1),  # overflow
     ((FAKE, FAKE, FAKE, FAKE, 2, 32768, 128, 128, 0.088, None, None), 2),  # B*H > 65535
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 64 * 16385, 128, 0.088, FAKE, None), 2),  # mask rows > 16384 blocks
+    ((FAKE, FAKE, FAKE, FAKE, 1, 1, 64 * 16385, 64, 0.088, FAKE, None), 2),   # the same at d = 64
     ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, 0.0, None, None), 1),     # sm_scale <= 0
     ((FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 128, float("nan"), None, None), 1),
 ])
