@@ -32,6 +32,8 @@ _lib.sa_attn_fwd.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_host.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_causal.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_attn_fwd_varlen.argtypes = [_P, _P, _P, _P, _I, _P, _I, _I, _F, _I, _P]
+_lib.sa_debug_varlen_groups.argtypes = [_I, _P, _I, _P]
+_lib.sa_debug_varlen_groups.restype = _I
 _lib.sa_attn_fwd_quantized.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]
 _lib.sa_debug_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P]
 _lib.sa_block_mask.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
@@ -186,6 +188,18 @@ def sa_attn_fwd_causal(q, k, v, sm_scale: float | None = None, block_mask=None, 
     _check(_lib.sa_attn_fwd_causal(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, N, d, scale, _ptr(m),
                                    _stream(q.device)), "sa_attn_fwd_causal")
     return o
+
+
+def sa_debug_varlen_groups(seqlens, H: int):
+    """The launch groups sa_attn_fwd_varlen forms for these lengths (host only): a list with
+    the group of each sequence, groups numbered in launch order."""
+    lens = [int(n) for n in seqlens]
+    arr = (ctypes.c_int * len(lens))(*lens)
+    out = (ctypes.c_int * len(lens))()
+    n = _lib.sa_debug_varlen_groups(len(lens), arr, int(H), out)
+    if n < 0:
+        raise ValueError("sa_debug_varlen_groups: bad arguments")
+    return list(out)
 
 
 def sa_attn_fwd_varlen(q, k, v, seqlens, H: int, sm_scale: float | None = None, causal: bool = False, out=None,

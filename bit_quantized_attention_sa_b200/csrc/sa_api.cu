@@ -384,6 +384,37 @@ static sa_status attn_fwd_host_pipeline(const void *q, const void *k, const void
     return SA_OK;
 }
 
+// Variable-length groups: sequences taken longest first (ord, a stable order); a group
+// runs as one prologue and one attention launch over heads padded to its longest sequence,
+// and takes the next sequence while the padded size stays within twice the group's own
+// (or below 2^20 padded token-heads, where the padding costs little) and its heads stay a
+// valid grid dimension.
+struct VarlenGroup {
+    int first, count;  // positions in ord
+    int64_t nmax;
+};
+static void varlen_groups(int nseq, const int *seqlens, int H, std::vector<int> &ord, std::vector<VarlenGroup> &groups)
+{
+    ord.resize(static_cast<size_t>(nseq));
+    std::iota(ord.begin(), ord.end(), 0);
+    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return seqlens[a] > seqlens[b]; });
+    groups.clear();
+    for (int g0 = 0; g0 < nseq;) {
+        const int64_t nmax = seqlens[ord[g0]], pmax = padded_len(nmax);
+        int64_t own = pmax;
+        int cnt = 1;
+        while (g0 + cnt < nseq) {
+            const int64_t own2 = own + padded_len(seqlens[ord[g0 + cnt]]), pad2 = int64_t(cnt + 1) * pmax;
+            if (pad2 > 2 * own2 && pad2 * H > (int64_t(1) << 20)) break;
+            if (int64_t(cnt + 1) * H > 65535) break;
+            own = own2;
+            ++cnt;
+        }
+        groups.push_back({g0, cnt, nmax});
+        g0 += cnt;
+    }
+}
+
 }  // namespace sa
 
 using namespace sa;
@@ -747,35 +778,14 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
         start[i + 1] = start[i] + seqlens[i];
     }
     if (start[nseq] > INT_MAX / 8 || int64_t(H) * start[nseq] > INT64_MAX / kD) return SA_ERR_INVALID_ARG;
-    // Groups: sequences taken longest first; a group runs as one prologue and one attention
-    // launch over heads padded to its longest sequence, and takes the next sequence while
-    // the padded size stays within twice the group's own (or below 2^20 padded
-    // token-heads, where the padding costs little).
-    std::vector<int> ord(static_cast<size_t>(nseq));
-    std::iota(ord.begin(), ord.end(), 0);
-    std::stable_sort(ord.begin(), ord.end(), [&](int a, int b) { return seqlens[a] > seqlens[b]; });
-    struct Group {
-        int first, count;
-        int64_t nmax;
-    };
-    std::vector<Group> groups;
+    std::vector<int> ord;
+    std::vector<VarlenGroup> groups;
+    varlen_groups(nseq, seqlens, H, ord, groups);
     size_t need = 0;
-    for (int g0 = 0; g0 < nseq;) {
-        const int64_t nmax = seqlens[ord[g0]], pmax = padded_len(nmax);
-        int64_t own = pmax;
-        int cnt = 1;
-        while (g0 + cnt < nseq) {
-            const int64_t own2 = own + padded_len(seqlens[ord[g0 + cnt]]), pad2 = int64_t(cnt + 1) * pmax;
-            if (pad2 > 2 * own2 && pad2 * H > (int64_t(1) << 20)) break;
-            if (int64_t(cnt + 1) * H > 65535) break;  // a group's heads are a grid dimension
-            own = own2;
-            ++cnt;
-        }
+    for (const VarlenGroup &g : groups) {
         Shape s;
-        if ((r = check_shape(cnt, H, int(nmax), d, &s)) != SA_OK) return r;
+        if ((r = check_shape(g.count, H, int(g.nmax), d, &s)) != SA_OK) return r;
         need = std::max(need, align256(ws_layout(s).total));
-        groups.push_back({g0, cnt, nmax});
-        g0 += cnt;
     }
     // device table after the largest group's workspace: the lengths in group order, then
     // the first row (of d elements) of every head in q, k, v and o
@@ -796,7 +806,7 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
     if ((r = upload_table(table.data(), tb, ws + need, st)) != SA_OK) return r;
     const int *dlens = reinterpret_cast<const int *>(ws + need);
     const int64_t *drows = reinterpret_cast<const int64_t *>(ws + need + lb);
-    for (const Group &g : groups) {
+    for (const VarlenGroup &g : groups) {
         Shape s;
         check_shape(g.count, H, int(g.nmax), d, &s);
         SeqTable t;
@@ -806,6 +816,19 @@ sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *
         if ((r = attn_fwd_device(q, k, v, o, s, sm_scale, nullptr, st, causal != 0, nullptr, t)) != SA_OK) return r;
     }
     return SA_OK;
+}
+
+int sa_debug_varlen_groups(int nseq, const int *seqlens, int H, int *group_of)
+{
+    if (nseq < 1 || !seqlens || !group_of || H < 1) return -1;
+    for (int i = 0; i < nseq; ++i)
+        if (seqlens[i] < 1) return -1;
+    std::vector<int> ord;
+    std::vector<VarlenGroup> groups;
+    varlen_groups(nseq, seqlens, H, ord, groups);
+    for (size_t g = 0; g < groups.size(); ++g)
+        for (int i = 0; i < groups[g].count; ++i) group_of[ord[size_t(groups[g].first + i)]] = int(g);
+    return int(groups.size());
 }
 
 sa_status sa_debug_qk_s32(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d,

@@ -154,6 +154,12 @@ sa_status sa_attn_fwd_causal(const void *q, const void *k, const void *v, void *
 sa_status sa_attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, int nseq, const int *seqlens,
                              int H, int d, float sm_scale, int causal, void *stream);
 
+/* Debug (host only, no CUDA call): the groups sa_attn_fwd_varlen forms for these lengths.
+ * group_of[i] (host array of nseq) receives the group of sequence i; groups are numbered
+ * in launch order (longest sequences first).  Returns the number of groups, or -1 on bad
+ * arguments (nseq < 1, H < 1, a null pointer or a length < 1). */
+int sa_debug_varlen_groups(int nseq, const int *seqlens, int H, int *group_of);
+
 /* Full forward on HOST buffers: q, k, v, o bf16 [B,H,N,d] and block_mask (or NULL) in host
  * memory, page-locked for the copies to overlap (pageable memory works but serialises).
  * The B*H heads are independent, so they are processed in chunks of consecutive heads
