@@ -166,11 +166,12 @@ int sa_debug_varlen_groups(int nseq, const int *seqlens, int H, int *group_of);
  * (one head first, then growing by one head per chunk up to about 64 MB of q, so that the
  * first upload, which nothing overlaps, is short): the upload of chunk c+1 and the
  * download of chunk c-1 run on two library-owned streams while chunk c runs sa_attn_fwd's
- * prologue and kernel on `stream`.  The call returns
- * after enqueueing; the work is complete when `stream` reaches the point after the call
- * (o is then filled), and q, k, v, o and block_mask must stay valid until then.  Device staging (two chunks) is library-owned, per device and
- * grow-only, like the workspace.  Calls for the same device from several host threads
- * are serialised.  Results are identical to sa_attn_fwd on the same inputs. */
+ * prologue and kernel on `stream`.  The call returns after enqueueing; the work is
+ * complete when `stream` reaches the point after the call (o is then filled), and q, k,
+ * v, o and block_mask must stay valid until then.  Device staging (two chunks) is
+ * library-owned, per device and grow-only, like the workspace.  Calls for the same device
+ * from several host threads are serialised.  Results are identical to sa_attn_fwd on the
+ * same inputs. */
 sa_status sa_attn_fwd_host(const void *q, const void *k, const void *v, void *o, int B, int H,
                            int N, int d, float sm_scale, const uint8_t *block_mask, void *stream);
 
